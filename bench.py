@@ -1,0 +1,376 @@
+"""Benchmark of the routed-expert MoE prefill layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one pass of the whole layer (route, group, gate/up decode-GEMM +
+SwiGLU, down decode-GEMM, combine) over one chunk of synthetic input, through
+the library's C ABI (rl_moe_prefill_ws).  Default workload: the 2,048-token
+chunk, H=2048, I=512, 512 experts, top-10, format Q2 (20,480 pairs).  The L2
+is flushed (a 256 MB device write) before every timed step; each step is timed
+with CUDA events on the launching stream.  The metric is routed pairs/s (the
+layer's ms per step is in ms_per_step).
+
+Multi-GPU: the layer does not shard (one GPU per layer call), so --gpus N runs
+N independent replicas, one process per GPU under torchrun; value is the pairs
+of all ranks divided by the slowest rank's time (scaling "weak").
+
+--impl reference times the float64 CPU oracle on host cores, each step a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_routed_expert_top_b200 import synth  # noqa: E402
+
+METRIC = "ms/layer & routed pairs/s at 2048 tok, 512 experts top-10; % of roofline"
+UNIT = "pairs/s"
+FLUSH_BYTES = 256 << 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def layer_model(wl, touched_experts: int):
+    """Algorithmic FLOPs and bytes of the layer and of its gate/up stage."""
+    P = wl.T * wl.k
+    flops = 6.0 * wl.H * wl.I * P
+    flops_gu = 4.0 * wl.H * wl.I * P
+    eb = synth.expert_bytes(wl.fmt, wl.H, wl.I)
+    bytes_w = touched_experts * eb
+    act = 2.0 * wl.T * wl.H + 4.0 * wl.T * wl.E + 4.0 * wl.T * wl.H
+    return dict(flops=flops, flops_gu=flops_gu, bytes=bytes_w + act,
+                bytes_gu=touched_experts * eb * 2 / 3 + 2.0 * wl.T * wl.H)
+
+
+def source_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def read_traffic(kernel_file):
+    """dram bytes per launch of the gate/up kernel from the committed ncu
+    summary, or None when the kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "gateup_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_sha256_16") != source_hash(kernel_file):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = str(gpu_index)
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.gpu], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def bench_reference(args, wl, world, rank):
+    """The float64 oracle as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    from oracle import moe_oracle as O
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    inp = synth.make_inputs(wl)
+    nb = synth.expert_bytes(wl.fmt, wl.H, wl.I)
+    blobs = [inp.blobs[e, :nb] for e in range(wl.E)]
+    ntok = 2 if wl.T >= 2 else 1
+    rng = np.random.default_rng(0)
+
+    def step():
+        toks = rng.integers(0, wl.T, ntok)
+        O.moe_prefill_tokens(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I, wl.k, toks)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = args.steps * ntok * wl.k / dt
+    sample = (f"{ntok} tokens x top-{wl.k} of the {wl.name} workload per step (routing, decode of "
+              f"the selected experts, float64 FFN, ordered combine), {args.steps} steps")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                       "format": synth.FMT_NAMES[wl.fmt]},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    """The oracle on a bounded sample of the workload, single process."""
+    from oracle import moe_oracle as O
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    inp = synth.make_inputs(wl)
+    nb = synth.expert_bytes(wl.fmt, wl.H, wl.I)
+    blobs = [inp.blobs[e, :nb] for e in range(wl.E)]
+    rng = np.random.default_rng(1)
+    done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        toks = rng.integers(0, wl.T, 2)
+        O.moe_prefill_tokens(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I, wl.k, toks)
+        done += 2
+    dt = time.perf_counter() - t0
+    return {"value": done * wl.k / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} tokens ({done * wl.k} pairs) of {wl.name}, {dt:.1f} s, float64"}
+
+
+def bench_ours(args, wl, world, rank, local):
+    import torch
+    import torch.distributed as dist
+    from bit_routed_expert_top_b200 import api
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+
+    inp = synth.make_inputs(wl)
+    x = torch.from_numpy(inp.x_bits.view(np.int16).copy()).to(dev)
+    logits = torch.from_numpy(inp.logits).to(dev)
+    blobs = torch.from_numpy(inp.blobs).to(dev)
+    table = api.expert_table(blobs, wl.E)
+    y = torch.empty((wl.T, wl.H), dtype=torch.float32, device=dev)
+    ws = api.alloc_workspace(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    P = wl.T * wl.k
+
+    def layer():
+        api.rl_moe_prefill_ws(x, logits, table, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws, stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        layer()
+    torch.cuda.synchronize()
+    bits = api.rl_moe_check_status(ws, stream)
+    if bits:
+        raise SystemExit(f"device status 0x{bits:x}: {api.rl_last_error()}")
+
+    # touched experts (for the byte count of the roofline)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+    w_ = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+    off = torch.empty(wl.E + 1, dtype=torch.int32, device=dev)
+    pl = torch.empty(P, dtype=torch.int32, device=dev)
+    pp = torch.empty(P, dtype=torch.int32, device=dev)
+    api.rl_moe_route(logits, wl.T, wl.E, wl.k, idx, w_, off, pl, pp, ws, stream)
+    counts = torch.diff(off).cpu().numpy()
+    touched = int((counts > 0).sum())
+
+    api.rl_moe_profile_enable(True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_ms = []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        layer()
+        ends[i].record(stream)
+        stage_ms.append(api.rl_moe_profile_read())
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    api.rl_moe_profile_enable(False)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    bits = api.rl_moe_check_status(ws, stream)
+    if bits:
+        raise SystemExit(f"device status 0x{bits:x}: {api.rl_last_error()}")
+
+    # end to end: pinned host inputs and output, copies inside the timed region
+    hx = torch.from_numpy(inp.x_bits.view(np.int16).copy()).pin_memory()
+    hl = torch.from_numpy(inp.logits.copy()).pin_memory()
+    hy = torch.empty((wl.T, wl.H), dtype=torch.float32).pin_memory()
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.warmup + args.steps):
+        flush.fill_(float(i))
+        if i >= args.warmup:
+            e_starts[i - args.warmup].record(stream)
+        x.copy_(hx, non_blocking=True)
+        logits.copy_(hl, non_blocking=True)
+        layer()
+        hy.copy_(y, non_blocking=True)
+        if i >= args.warmup:
+            e_ends[i - args.warmup].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    model = layer_model(wl, touched)
+    gu_ms = statistics.mean(s["gateup"] for s in stage_ms)
+    ms_step = total_ms / args.steps
+    achieved_tf = model["flops_gu"] / (gu_ms * 1e-3) / 1e12
+    peak_tf = peaks["bf16_tflops"]
+    t_roof_ms = max(model["flops"] / (peaks["bf16_tflops"] * 1e12),
+                    model["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    kernel_file = os.path.join(ROOT, "bit_routed_expert_top_b200", "csrc", "gemm_tc.cuh")
+    traffic = read_traffic(kernel_file)
+    value = world * args.steps * P / (total_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                   "format": synth.FMT_NAMES[wl.fmt], "pairs": P, "touched_experts": touched,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed by a 256 MB device write before every timed step",
+                   "arithmetic": "fp16 decoded weights and activations, fp32 accumulate, fp32 y"},
+        "roofline": {"bound": "tensor", "kernel": "gate/up decode-GEMM + SwiGLU",
+                     "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved_tf / peak_tf, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 dense (fp16 same rate), burst"},
+        "layer_roofline": {"t_roof_ms": t_roof_ms, "t_meas_ms": ms_step,
+                           "frac": t_roof_ms / ms_step,
+                           "tflops": model["flops"] / (ms_step * 1e-3) / 1e12,
+                           "algorithmic_bytes": model["bytes"]},
+        "stages_ms": {k: statistics.mean(s[k] for s in stage_ms) for k in stage_ms[0]},
+        "routed_tokens_per_s": world * args.steps * wl.T / (total_ms * 1e-3),
+        "e2e": {"value": world * args.steps * P / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": int(x.numel() * 2 + logits.numel() * 4),
+                "d2h_bytes_per_step": int(y.numel() * 4)},
+        "gpu_launches": args.steps * api.rl_moe_launches_per_call(),
+        "clocks": clocks,
+        "wall_s_timed_region": wall,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=synth.WORKLOADS[synth.HEADLINE].name,
+                    choices=[w.name for w in synth.WORKLOADS])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    wl = next(w for w in synth.WORKLOADS if w.name == args.workload)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        bench_reference(args, wl, world, rank)
+    else:
+        bench_ours(args, wl, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

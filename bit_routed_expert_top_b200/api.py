@@ -1,0 +1,187 @@
+"""Python binding of librl_moe.so (argument marshalling only).
+
+Every function has the name of the C entry point it calls (include/rl_moe.h)
+and takes torch tensors for device buffers; all work runs in the library's
+CUDA kernels.  There is no CPU path: if the shared library is missing or no
+CUDA device is present, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+FMT_Q1 = 1
+FMT_Q2 = 2
+RL_OK = 0
+STATUS_NAMES = {-1: "RL_ERR_INVALID_ARG", -2: "RL_ERR_UNSUPPORTED", -3: "RL_ERR_CUDA",
+                -4: "RL_ERR_DEVICE_STATUS"}
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librl_moe.so")
+
+# Every symbol include/rl_moe.h declares, with its ctypes signature.
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "rl_moe_block_bytes": (_sz, [_i]),
+    "rl_moe_expert_bytes": (_sz, [_i, _i, _i]),
+    "rl_moe_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "rl_moe_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp]),
+    "rl_moe_prefill_ws": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "rl_moe_route": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "rl_moe_check_status": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_uint)]),
+    "rl_moe_profile_enable": (_i, [_i]),
+    "rl_moe_profile_read": (_i, [ctypes.POINTER(ctypes.c_float), _i]),
+    "rl_moe_profile_stage_name": (ctypes.c_char_p, [_i]),
+    "rl_moe_launches_per_call": (_i, []),
+    "rl_last_error": (ctypes.c_char_p, []),
+}
+# Not in the public header: selects the CUDA-core decode-GEMMs for stage-by-
+# stage cross-checks of the tensor-core kernels.
+DEBUG_SIGNATURES = {
+    "rl_moe_debug_set_gemm": (_i, [_i]),
+}
+
+_lib = None
+
+
+class RlMoeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the shared library (once).  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"librl_moe.so not found at {path}; build it with "
+                           "python bit_routed_expert_top_b200/csrc/build.py")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in {**SIGNATURES, **DEBUG_SIGNATURES}.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != RL_OK:
+        raise RlMoeError(rc, load().rl_last_error().decode(errors="replace"))
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not isinstance(t, int) and not t.is_cuda:
+            raise ValueError("device buffers must be CUDA tensors")
+
+
+def expert_table(blobs, E: int | None = None):
+    """Host array of expert pointers: from a CUDA uint8 tensor [E, stride]
+    (expert e at row e) or a sequence of CUDA tensors / integer addresses."""
+    if isinstance(blobs, torch.Tensor):
+        _need_cuda(blobs)
+        E = blobs.shape[0] if E is None else E
+        base, stride = blobs.data_ptr(), blobs.stride(0) * blobs.element_size()
+        ptrs = [base + e * stride for e in range(E)]
+    else:
+        ptrs = [_ptr(b) for b in blobs]
+    arr = (ctypes.c_void_p * len(ptrs))(*ptrs)
+    return arr
+
+
+def rl_moe_block_bytes(fmt: int) -> int:
+    return load().rl_moe_block_bytes(fmt)
+
+
+def rl_moe_expert_bytes(fmt: int, H: int, I: int) -> int:
+    return load().rl_moe_expert_bytes(fmt, H, I)
+
+
+def rl_moe_workspace_bytes(fmt: int, T: int, H: int, I: int, E: int, k: int) -> int:
+    n = load().rl_moe_workspace_bytes(fmt, T, H, I, E, k)
+    if n == 0:
+        raise RlMoeError(-1, load().rl_last_error().decode(errors="replace"))
+    return n
+
+
+def alloc_workspace(fmt, T, H, I, E, k, device=None) -> torch.Tensor:
+    n = rl_moe_workspace_bytes(fmt, T, H, I, E, k)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def rl_moe_prefill(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, stream=None):
+    _need_cuda(x, router_logits, y)
+    table = expert_blobs if isinstance(expert_blobs, ctypes.Array) else expert_table(expert_blobs, E)
+    _check(load().rl_moe_prefill(_ptr(x), _ptr(router_logits), ctypes.cast(table, ctypes.c_void_p),
+                                 fmt, T, H, I, E, k, _ptr(y), _stream(stream)))
+
+
+def rl_moe_prefill_ws(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, workspace,
+                      stream=None):
+    _need_cuda(x, router_logits, y, workspace)
+    table = expert_blobs if isinstance(expert_blobs, ctypes.Array) else expert_table(expert_blobs, E)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().rl_moe_prefill_ws(_ptr(x), _ptr(router_logits), ctypes.cast(table, ctypes.c_void_p),
+                                    fmt, T, H, I, E, k, _ptr(y), _ptr(workspace), nbytes,
+                                    _stream(stream)))
+
+
+def rl_moe_route(router_logits, T, E, k, topk_idx, topk_w, offsets, pair_list, pair_pos,
+                 workspace, stream=None):
+    _need_cuda(router_logits, topk_idx, topk_w, offsets, pair_list, pair_pos, workspace)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().rl_moe_route(_ptr(router_logits), T, E, k, _ptr(topk_idx), _ptr(topk_w),
+                               _ptr(offsets), _ptr(pair_list), _ptr(pair_pos), _ptr(workspace),
+                               nbytes, _stream(stream)))
+
+
+def rl_moe_check_status(workspace, stream=None) -> int:
+    """Returns the device status bits (0 = fine); raises on a CUDA error."""
+    bits = ctypes.c_uint(0)
+    rc = load().rl_moe_check_status(_ptr(workspace), _stream(stream), ctypes.byref(bits))
+    if rc not in (RL_OK, -4):
+        _check(rc)
+    return bits.value
+
+
+def rl_moe_profile_enable(on: bool = True):
+    _check(load().rl_moe_profile_enable(1 if on else 0))
+
+
+def rl_moe_profile_read() -> dict:
+    n = 5
+    buf = (ctypes.c_float * n)()
+    _check(load().rl_moe_profile_read(buf, n))
+    return {load().rl_moe_profile_stage_name(i).decode(): float(buf[i]) for i in range(n)}
+
+
+def rl_moe_launches_per_call() -> int:
+    return load().rl_moe_launches_per_call()
+
+
+def rl_last_error() -> str:
+    return load().rl_last_error().decode(errors="replace")
+
+
+def debug_set_gemm(which: str):
+    """'tc' (tensor cores, the default) or 'simt' (CUDA cores, cross-check)."""
+    _check(load().rl_moe_debug_set_gemm({"tc": 0, "simt": 1}[which]))

@@ -1,0 +1,116 @@
+// common.cuh - shared definitions of the B200 routed-expert MoE kernels.
+//
+// Block formats (stand-ins for IQ2_XS / IQ1_M; the Red Lite pages do not
+// print those grids): 256 values per block along K, fp16 scale d, eight 3-bit
+// sub-scales s (one per 32 values).
+//   Q2, 69 B: w = d(2s+1)(2u-3), 2-bit code u;  Q1, 38 B: w = d(2s+1)((2b-1)+delta).
+// Expert blob: gate [I rows of K=H] | up [I rows] | down [H rows of K=I].
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "../../include/rl_moe.h"
+
+namespace rl {
+
+constexpr int kBlockVals = 256;
+constexpr int kSubVals = 32;
+constexpr int kQ2Bytes = 69;
+constexpr int kQ1Bytes = 38;
+constexpr int kMaxE = RL_MAX_EXPERTS;
+
+// Rows of one tensor-core M tile; also the row slab of a work unit.
+constexpr int kSlabRows = 128;
+
+template <int FMT> struct Fmt;
+// Q2: 2-bit codes, 4 codes per byte, 16 codes per 32-bit word.
+template <> struct Fmt<RL_FMT_Q2> {
+  static constexpr int kBytes = kQ2Bytes;
+  static constexpr int kCodeOff = 5;       // first code byte
+  static constexpr int kBits = 2;
+  static constexpr int kPerByte = 4;
+  static constexpr int kGroup = 16;        // values per code word = K-permutation group
+};
+// Q1: 1-bit codes, 8 per byte, 32 per word; byte 5 holds the shift flags.
+template <> struct Fmt<RL_FMT_Q1> {
+  static constexpr int kBytes = kQ1Bytes;
+  static constexpr int kCodeOff = 6;
+  static constexpr int kBits = 1;
+  static constexpr int kPerByte = 8;
+  static constexpr int kGroup = 32;
+};
+
+// K permutation shared by the decoded weights (A operand) and the staged
+// activations (B operand).  The decoder turns one 32-bit code word
+// (kGroup consecutive values) into kGroup/2 fp16x2 words; word c, half h
+// holds the value pi(2c+h) of the group, with
+//     pi(i) = (i >> 2) + kPerByte * (i & 3).
+// A dot product is unchanged by a K permutation applied to both operands, so
+// x (and h for the down projection) are stored with the same permutation:
+// position i of a group holds natural value pi(i).
+template <int FMT>
+__host__ __device__ __forceinline__ int perm_value(int i) {
+  return (i >> 2) + Fmt<FMT>::kPerByte * (i & 3);
+}
+// Inverse: natural value v of a group sits at position perm_pos(v).
+template <int FMT>
+__host__ __device__ __forceinline__ int perm_pos(int v) {
+  return 4 * (v % Fmt<FMT>::kPerByte) + v / Fmt<FMT>::kPerByte;
+}
+template <int FMT>
+__host__ __device__ __forceinline__ int perm_pos_k(int k) {
+  constexpr int G = Fmt<FMT>::kGroup;
+  return (k / G) * G + perm_pos<FMT>(k % G);
+}
+
+// Per-call expert pointer table, passed BY VALUE in the kernel parameters so
+// that a later call cannot change the table an enqueued call reads (the
+// Red Lite dev72 page, section 1, traces a wrong-output bug to tables kept
+// in shared buffers and rewritten by the next row's encode).
+struct ExpertTable {
+  const uint8_t* p[kMaxE];
+};
+
+struct Dims {
+  int T, H, I, E, k, fmt;
+  int P;          // T * k pairs
+  int W;          // ceil(T / 32) bitmap words per expert
+  int nbH, nbI;   // blocks per row of gate/up (K=H) and down (K=I)
+  int bb;         // bytes per block
+  int slabs_gu;   // ceil(I / 128) row slabs of gate (and of up)
+  int slabs_dn;   // ceil(H / 128) row slabs of down
+  int mt_dn;      // down slabs per work unit
+  int groups_dn;  // ceil(slabs_dn / mt_dn)
+  int nt_gu;      // max pairs per gate/up work unit
+  int nt_dn;      // max pairs per down work unit
+  int max_units_gu, max_units_dn;
+};
+
+// Device pieces carved from the workspace (or caller buffers for rl_moe_route).
+struct Work {
+  unsigned* status;      // [0]: RL_DEV_* bits of the latest call
+  int* idx;              // [P] expert of pair t*k+j
+  float* pw;             // [P] routing weight p_{t,j}
+  unsigned* bitmap;      // [E][W] bit b of word w: token 32w+b chose expert e
+  uint16_t* jslot;       // [E][T] slot j of token t for expert e (valid where bit set)
+  int* offsets;          // [E+1]
+  int* pair_list;        // [P] grouped by expert, ascending token
+  int* pair_pos;         // [P] inverse
+  int* counters;         // [0] gate/up units, [1] down units
+  int4* units_gu;        // {expert, slab, first grouped position, pairs}
+  int4* units_dn;        // {expert, slab group, first grouped position, pairs}
+  __half* x16;           // [T][H] x as fp16, K-permuted per group
+  __half* h16;           // [P][I] h, grouped order, K-permuted per group
+  __half* o16;           // [P][H] o, pair-id order
+};
+
+__device__ __forceinline__ void set_status(unsigned* st, unsigned bits) {
+  atomicOr(st, bits);
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint32_t bits16) {
+  return __half2float(__ushort_as_half((unsigned short)bits16));
+}
+
+}  // namespace rl

@@ -1,0 +1,321 @@
+// rl_moe.cu - host side of librl_moe.so: argument checks, workspace layout,
+// kernel launches and the C ABI declared in include/rl_moe.h.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "route_group.cuh"
+
+namespace {
+
+thread_local std::string t_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(RL_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Work-unit shapes of the decode-GEMM stages (see gemm_tc.cuh).
+constexpr int kNtGateUp = rl::tc::kNtGu;
+constexpr int kNtDown = rl::tc::kNtDn;
+constexpr int kMtDown = rl::tc::kMtDn;
+
+struct Layout {
+  size_t status, idx, pw, bitmap, jslot, offsets, pair_list, pair_pos, counters,
+      units_gu, units_dn, x16, h16, o16, total;
+};
+
+int check_dims(int fmt, int T, int H, int I, int E, int k) {
+  if (fmt != RL_FMT_Q1 && fmt != RL_FMT_Q2) return fail(RL_ERR_INVALID_ARG, "unknown fmt %d", fmt);
+  if (T < 0) return fail(RL_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (E < 1) return fail(RL_ERR_INVALID_ARG, "E=%d < 1", E);
+  if (k < 1 || k > E) return fail(RL_ERR_INVALID_ARG, "k=%d outside [1, E=%d]", k, E);
+  if (H <= 0 || I <= 0) return fail(RL_ERR_INVALID_ARG, "H=%d, I=%d must be positive", H, I);
+  if (E > RL_MAX_EXPERTS) return fail(RL_ERR_UNSUPPORTED, "E=%d > %d", E, RL_MAX_EXPERTS);
+  if (H % 32 || I % 32 || H > RL_MAX_DIM || I > RL_MAX_DIM)
+    return fail(RL_ERR_UNSUPPORTED, "H=%d, I=%d must be multiples of 32 in [32, %d]", H, I, RL_MAX_DIM);
+  if ((long long)T * k > RL_MAX_PAIRS)
+    return fail(RL_ERR_UNSUPPORTED, "T*k=%lld > %d", (long long)T * k, RL_MAX_PAIRS);
+  return RL_OK;
+}
+
+int plan(int fmt, int T, int H, int I, int E, int k, rl::Dims* d, Layout* L) {
+  const int rc = check_dims(fmt, T, H, I, E, k);
+  if (rc != RL_OK) return rc;
+  d->T = T; d->H = H; d->I = I; d->E = E; d->k = k; d->fmt = fmt;
+  d->P = T * k;
+  d->W = (T + 31) / 32;
+  d->nbH = (H + rl::kBlockVals - 1) / rl::kBlockVals;
+  d->nbI = (I + rl::kBlockVals - 1) / rl::kBlockVals;
+  d->bb = fmt == RL_FMT_Q2 ? rl::kQ2Bytes : rl::kQ1Bytes;
+  d->slabs_gu = (I + rl::kSlabRows - 1) / rl::kSlabRows;
+  d->slabs_dn = (H + rl::kSlabRows - 1) / rl::kSlabRows;
+  d->mt_dn = kMtDown;
+  d->groups_dn = (d->slabs_dn + kMtDown - 1) / kMtDown;
+  d->nt_gu = kNtGateUp;
+  d->nt_dn = kNtDown;
+  d->max_units_gu = d->slabs_gu * (E + (d->P + kNtGateUp - 1) / kNtGateUp);
+  d->max_units_dn = d->groups_dn * (E + (d->P + kNtDown - 1) / kNtDown);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = align_up(o + bytes, 256); return at; };
+  L->status = take(256);
+  L->idx = take((size_t)d->P * 4);
+  L->pw = take((size_t)d->P * 4);
+  L->bitmap = take((size_t)E * d->W * 4);
+  L->jslot = take((size_t)E * T * 2);
+  L->offsets = take((size_t)(E + 1) * 4);
+  L->pair_list = take((size_t)d->P * 4);
+  L->pair_pos = take((size_t)d->P * 4);
+  L->counters = take(64);
+  L->units_gu = take((size_t)d->max_units_gu * 16);
+  L->units_dn = take((size_t)d->max_units_dn * 16);
+  L->x16 = take((size_t)T * H * 2);
+  L->h16 = take((size_t)d->P * I * 2);
+  L->o16 = take((size_t)d->P * H * 2);
+  L->total = o;
+  return RL_OK;
+}
+
+rl::Work carve(void* ws, const Layout& L) {
+  char* b = static_cast<char*>(ws);
+  rl::Work w;
+  w.status = reinterpret_cast<unsigned*>(b + L.status);
+  w.idx = reinterpret_cast<int*>(b + L.idx);
+  w.pw = reinterpret_cast<float*>(b + L.pw);
+  w.bitmap = reinterpret_cast<unsigned*>(b + L.bitmap);
+  w.jslot = reinterpret_cast<uint16_t*>(b + L.jslot);
+  w.offsets = reinterpret_cast<int*>(b + L.offsets);
+  w.pair_list = reinterpret_cast<int*>(b + L.pair_list);
+  w.pair_pos = reinterpret_cast<int*>(b + L.pair_pos);
+  w.counters = reinterpret_cast<int*>(b + L.counters);
+  w.units_gu = reinterpret_cast<int4*>(b + L.units_gu);
+  w.units_dn = reinterpret_cast<int4*>(b + L.units_dn);
+  w.x16 = reinterpret_cast<__half*>(b + L.x16);
+  w.h16 = reinterpret_cast<__half*>(b + L.h16);
+  w.o16 = reinterpret_cast<__half*>(b + L.o16);
+  return w;
+}
+
+// ---- stage timing ----------------------------------------------------------
+constexpr int kStages = 5;
+const char* kStageNames[kStages] = {"route", "group", "gateup", "down", "combine"};
+bool g_prof = false;
+cudaEvent_t g_ev[kStages + 1];
+bool g_ev_made = false;
+bool g_ev_recorded = false;
+
+inline void mark(int i, cudaStream_t s) {
+  if (g_prof) cudaEventRecord(g_ev[i], s);
+}
+
+// Which decode-GEMM implementation runs (0: tensor cores, 1: CUDA cores).
+int g_gemm = 0;
+
+template <int FMT>
+int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
+               const rl::Work& w, float* y, cudaStream_t s) {
+  mark(0, s);
+  rl::route_kernel<FMT><<<d.W, 1024, 0, s>>>(logits, static_cast<const uint16_t*>(x), d, w);
+  mark(1, s);
+  rl::group_kernel<<<1, 1024, 0, s>>>(d, w, 1);
+  mark(2, s);
+  if (g_gemm == 1) {
+    rl::gateup_simt_kernel<FMT><<<d.max_units_gu, 256, 0, s>>>(d, w, tab);
+    mark(3, s);
+    rl::down_simt_kernel<FMT><<<d.max_units_dn, 256, 0, s>>>(d, w, tab);
+  } else {
+    const int rc = rl::tc::launch_gateup<FMT>(d, w, tab, s);
+    if (rc != RL_OK) return rc;
+    mark(3, s);
+    const int rc2 = rl::tc::launch_down<FMT>(d, w, tab, s);
+    if (rc2 != RL_OK) return rc2;
+  }
+  mark(4, s);
+  rl::combine_kernel<<<dim3(d.T, (d.H + 1023) / 1024), 256, 0, s>>>(d, w.pw, w.o16, y);
+  mark(5, s);
+  if (g_prof) g_ev_recorded = true;
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return RL_OK;
+}
+
+int fill_table(const void* const* blobs, int E, rl::ExpertTable* tab) {
+  if (!blobs) return fail(RL_ERR_INVALID_ARG, "expert_blobs is NULL");
+  for (int e = 0; e < E; ++e) {
+    const void* p = blobs[e];
+    if (!p) return fail(RL_ERR_INVALID_ARG, "expert_blobs[%d] is NULL", e);
+    if (reinterpret_cast<uintptr_t>(p) % 16)
+      return fail(RL_ERR_INVALID_ARG, "expert_blobs[%d] is not 16-byte aligned", e);
+    tab->p[e] = static_cast<const uint8_t*>(p);
+  }
+  for (int e = E; e < rl::kMaxE; ++e) tab->p[e] = nullptr;
+  return RL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t rl_moe_block_bytes(int fmt) {
+  return fmt == RL_FMT_Q2 ? rl::kQ2Bytes : fmt == RL_FMT_Q1 ? rl::kQ1Bytes : 0;
+}
+
+size_t rl_moe_expert_bytes(int fmt, int H, int I) {
+  const size_t bb = rl_moe_block_bytes(fmt);
+  if (!bb || H <= 0 || I <= 0) return 0;
+  const size_t nbH = (H + 255) / 256, nbI = (I + 255) / 256;
+  return (2 * (size_t)I * nbH + (size_t)H * nbI) * bb;
+}
+
+size_t rl_moe_workspace_bytes(int fmt, int T, int H, int I, int E, int k) {
+  rl::Dims d;
+  Layout L;
+  if (plan(fmt, T, H, I, E, k, &d, &L) != RL_OK) return 0;
+  return L.total;
+}
+
+int rl_moe_prefill_ws(const void* x, const float* router_logits, const void* const* expert_blobs,
+                      int fmt, int T, int H, int I, int E, int k, float* y, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  rl::Dims d;
+  Layout L;
+  int rc = plan(fmt, T, H, I, E, k, &d, &L);
+  if (rc != RL_OK) return rc;
+  if (T == 0) return RL_OK;
+  if (!x || !router_logits || !y || !workspace)
+    return fail(RL_ERR_INVALID_ARG, "NULL x, router_logits, y or workspace");
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(y) % 16 ||
+      reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(RL_ERR_INVALID_ARG, "x and y must be 16-byte aligned, workspace 256-byte aligned");
+  if (ws_bytes < L.total)
+    return fail(RL_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, L.total);
+  static thread_local rl::ExpertTable tab;
+  rc = fill_table(expert_blobs, E, &tab);
+  if (rc != RL_OK) return rc;
+  const rl::Work w = carve(workspace, L);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return fmt == RL_FMT_Q2 ? launch_all<RL_FMT_Q2>(x, router_logits, tab, d, w, y, s)
+                          : launch_all<RL_FMT_Q1>(x, router_logits, tab, d, w, y, s);
+}
+
+int rl_moe_prefill(const void* x, const float* router_logits, const void* const* expert_blobs,
+                   int fmt, int T, int H, int I, int E, int k, float* y, void* stream) {
+  rl::Dims d;
+  Layout L;
+  int rc = plan(fmt, T, H, I, E, k, &d, &L);
+  if (rc != RL_OK) return rc;
+  if (T == 0) return RL_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, L.total, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+  rc = rl_moe_prefill_ws(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, ws, L.total, stream);
+  e = cudaFreeAsync(ws, s);
+  if (rc != RL_OK) return rc;
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+  return RL_OK;
+}
+
+int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx, float* topk_w,
+                 int* offsets, int* pair_list, int* pair_pos, void* workspace, size_t ws_bytes,
+                 void* stream) {
+  rl::Dims d;
+  Layout L;
+  int rc = plan(RL_FMT_Q2, T, 32, 32, E, k, &d, &L);
+  if (rc != RL_OK) return rc;
+  if (T == 0) return RL_OK;
+  if (!router_logits || !topk_idx || !topk_w || !offsets || !pair_list || !pair_pos || !workspace)
+    return fail(RL_ERR_INVALID_ARG, "NULL pointer argument");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(RL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < L.total)
+    return fail(RL_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, L.total);
+  rl::Work w = carve(workspace, L);
+  w.idx = topk_idx;
+  w.pw = topk_w;
+  w.offsets = offsets;
+  w.pair_list = pair_list;
+  w.pair_pos = pair_pos;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rl::route_kernel<RL_FMT_Q2><<<d.W, 1024, 0, s>>>(router_logits, nullptr, d, w);
+  rl::group_kernel<<<1, 1024, 0, s>>>(d, w, 0);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return RL_OK;
+}
+
+int rl_moe_check_status(void* workspace, void* stream, unsigned* bits_out) {
+  if (!workspace) return fail(RL_ERR_INVALID_ARG, "NULL workspace");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned bits = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  e = cudaMemcpy(&bits, workspace, sizeof bits, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+  e = cudaMemset(workspace, 0, sizeof bits);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status)");
+  if (bits_out) *bits_out = bits;
+  if (bits)
+    return fail(RL_ERR_DEVICE_STATUS, "device status 0x%x:%s%s%s", bits,
+                bits & RL_DEV_UNIT_OVERFLOW ? " work-list overflow" : "",
+                bits & RL_DEV_WAIT_TIMEOUT ? " bounded wait timed out" : "",
+                bits & RL_DEV_BAD_GROUPING ? " grouped pair count != T*k" : "");
+  return RL_OK;
+}
+
+int rl_moe_profile_enable(int on) {
+  if (on && !g_ev_made) {
+    for (int i = 0; i <= kStages; ++i) {
+      const cudaError_t e = cudaEventCreate(&g_ev[i]);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+    }
+    g_ev_made = true;
+  }
+  g_prof = on != 0;
+  g_ev_recorded = false;
+  return RL_OK;
+}
+
+int rl_moe_profile_read(float* stage_ms, int n) {
+  if (!g_ev_made || !g_ev_recorded) return fail(RL_ERR_INVALID_ARG, "no profiled call recorded");
+  cudaError_t e = cudaEventSynchronize(g_ev[kStages]);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+  for (int i = 0; i < kStages && i < n; ++i) {
+    e = cudaEventElapsedTime(&stage_ms[i], g_ev[i], g_ev[i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+  }
+  return RL_OK;
+}
+
+const char* rl_moe_profile_stage_name(int i) {
+  return (i >= 0 && i < kStages) ? kStageNames[i] : "";
+}
+
+int rl_moe_launches_per_call(void) { return kStages; }
+
+int rl_moe_debug_set_gemm(int which) {
+  if (which != 0 && which != 1) return fail(RL_ERR_INVALID_ARG, "gemm %d", which);
+  g_gemm = which;
+  return RL_OK;
+}
+
+const char* rl_last_error(void) { return t_err.c_str(); }
+
+}  // extern "C"

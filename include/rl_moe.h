@@ -1,0 +1,152 @@
+/*
+ * rl_moe.h - C ABI of the B200 (sm_100a) routed-expert MoE prefill layer.
+ *
+ * One call computes, for a chunk of T tokens, the routed-expert layer that the
+ * Red Lite milestone pages profile ("Red Lite dev72 - bounded verify,
+ * profiling", section 4, second profile: 2,048 tokens, 512 experts, 20,480
+ * token/expert pairs; "Red Lite dev75 - --kv f16, faster prompt ingestion",
+ * section 2: the routed experts are bound by decoding their weights):
+ *
+ *   1. route    per token, the k largest router logits (selection order
+ *               j = 0..k-1: descending fp32 value, equal values to the lower
+ *               expert index) and p_j = softmax over those k
+ *               (dev72 section 1: router selection per row; section 3:
+ *               near-ties flip the routing, so selection is exact fp32);
+ *   2. group    the T*k pairs (pair id t*k+j) grouped by expert, ascending
+ *               token inside an expert (dev75 section 2: the experts work on
+ *               slices of their pairs; dev72 section 4: ~40 pairs/expert);
+ *   3. gate/up  g = W_gate x, u = W_up x with the weights decoded on the fly
+ *               from 1-2-bit blocks, h = silu(g) * u (SwiGLU);
+ *   4. down     o = W_down h, decoded the same way;
+ *   5. combine  y[t] = sum_j p_j o_{t,j}, added in selection order
+ *               (dev75 section 3: the MoE tail sums in selection order).
+ *
+ * Weight formats (stand-ins for IQ2_XS / IQ1_M, whose grids the pages do not
+ * print).  A block holds 256 consecutive values of one row along K:
+ *   RL_FMT_Q2, 69 bytes: [0,2) fp16 d (little endian); [2,5) 24-bit LE word,
+ *     sub-scale s_i of values 32i..32i+31 in bits 3i..3i+2; [5,69) 2-bit codes,
+ *     value v in byte 5+v/4 at bits 2(v%4); w = d(2s+1)(2u-3).
+ *   RL_FMT_Q1, 38 bytes: [0,2) d; [2,5) sub-scales; byte 5 bit i = shift flag
+ *     of sub-block i (0: -1/8, 1: +1/8); [6,38) 1-bit codes, value v in byte
+ *     6+v/8 at bit v%8; w = d(2s+1)((2b-1) + delta).
+ * Expert blob: W_gate [I rows] | W_up [I rows] | W_down [H rows]; a row of a
+ * matrix with K columns is ceil(K/256) consecutive blocks (values past K are
+ * ignored).  Bytes per expert: rl_moe_expert_bytes().
+ *
+ * Arithmetic: decoded weights are rounded once to fp16, x (bf16) is converted
+ * to fp16, products accumulate in fp32 on the tensor cores, h is stored as
+ * fp16, o as fp16, the combine runs in fp32.  y is fp32.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are CUDA global memory on the current device; host
+ *     pointers are ordinary host memory.  The caller owns every buffer; the
+ *     library keeps no pointer after the call returns.
+ *   - Work is enqueued on `stream` (0 = legacy default stream) and the call
+ *     returns after enqueue.  Results are ready when the stream reaches them.
+ *   - A negative return is an rl_status; rl_last_error() gives a message.
+ *     Kernels never trap: problems detected on the device set a status word
+ *     in the workspace, read by rl_moe_check_status().
+ */
+#ifndef RL_MOE_H
+#define RL_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { RL_FMT_Q1 = 1, RL_FMT_Q2 = 2 } rl_fmt;
+
+typedef enum {
+  RL_OK = 0,
+  RL_ERR_INVALID_ARG = -1,   /* null pointer, bad size, misaligned blob, short workspace */
+  RL_ERR_UNSUPPORTED = -2,   /* a shape outside the limits below                       */
+  RL_ERR_CUDA = -3,          /* a CUDA runtime call failed (message has the CUDA error) */
+  RL_ERR_DEVICE_STATUS = -4  /* rl_moe_check_status: a kernel reported a problem        */
+} rl_status;
+
+/* Limits: 1 <= k <= E <= RL_MAX_EXPERTS; H and I multiples of 32 in
+ * [32, RL_MAX_DIM]; 0 <= T and T*k <= RL_MAX_PAIRS. */
+#define RL_MAX_EXPERTS 1024
+#define RL_MAX_DIM 8192
+#define RL_MAX_PAIRS (1 << 24)
+
+/* Device status bits (rl_moe_check_status). */
+#define RL_DEV_UNIT_OVERFLOW 0x1u  /* a work list did not fit its reserved space  */
+#define RL_DEV_WAIT_TIMEOUT  0x2u  /* a bounded wait inside a kernel gave up      */
+#define RL_DEV_BAD_GROUPING  0x4u  /* the grouped pair count differed from T*k   */
+
+/* Bytes of one block of `fmt` (69 or 38); 0 for an unknown format. */
+size_t rl_moe_block_bytes(int fmt);
+
+/* Bytes of one expert blob (gate, up, down); 0 on a bad argument. */
+size_t rl_moe_expert_bytes(int fmt, int H, int I);
+
+/* Workspace bytes rl_moe_prefill_ws needs for these sizes (256-byte aligned
+ * pieces inside); 0 on a bad argument. */
+size_t rl_moe_workspace_bytes(int fmt, int T, int H, int I, int E, int k);
+
+/*
+ * The whole layer.
+ *   x             device, bf16 [T, H] row-major (raw bf16 bit patterns).
+ *   router_logits device, fp32 [T, E] row-major; finite values.
+ *   expert_blobs  HOST array of E device pointers, one blob per expert, each
+ *                 16-byte aligned and rl_moe_expert_bytes(fmt, H, I) long.
+ *                 The table is copied by value into the launches, so the
+ *                 caller may change or free the host array once the call
+ *                 returns (the blobs themselves must live until the stream
+ *                 has run the call).
+ *   y             device, fp32 [T, H] row-major, overwritten.
+ * Draws its workspace from the stream-ordered allocator (cudaMallocAsync on
+ * `stream`) and frees it stream-ordered; device status is then not readable,
+ * use rl_moe_prefill_ws for that.  T = 0 is a no-op.
+ */
+int rl_moe_prefill(const void* x, const float* router_logits,
+                   const void* const* expert_blobs, int fmt, int T, int H, int I,
+                   int E, int k, float* y, void* stream);
+
+/* Same, with a caller-owned device workspace of at least
+ * rl_moe_workspace_bytes() bytes, 256-byte aligned.  Calls that share a
+ * workspace must be ordered on one stream. */
+int rl_moe_prefill_ws(const void* x, const float* router_logits,
+                      const void* const* expert_blobs, int fmt, int T, int H,
+                      int I, int E, int k, float* y, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/*
+ * Steps 1-2 alone (parity/debug export).  Outputs, all device memory:
+ *   topk_idx int32 [T, k], topk_w fp32 [T, k]  (selection order)
+ *   offsets  int32 [E + 1]                     (exclusive prefix of counts)
+ *   pair_list int32 [T*k]: pair ids grouped by expert, ascending token
+ *   pair_pos  int32 [T*k]: inverse of pair_list
+ * workspace: rl_moe_workspace_bytes(RL_FMT_Q2, T, 32, 32, E, k) bytes suffice.
+ */
+int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx,
+                 float* topk_w, int* offsets, int* pair_list, int* pair_pos,
+                 void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronizes `stream`, reads and clears the device status word of
+ * `workspace`; returns RL_OK, or RL_ERR_DEVICE_STATUS with the bits in
+ * *bits_out (may be NULL) and the message in rl_last_error(). */
+int rl_moe_check_status(void* workspace, void* stream, unsigned* bits_out);
+
+/* Stage timing: when enabled, rl_moe_prefill[_ws] records CUDA events on its
+ * stream around each kernel; rl_moe_profile_read() synchronizes on the last
+ * events and writes up to n stage times in milliseconds (route, group,
+ * gate/up, down, combine) plus names via rl_moe_profile_stage_name(). */
+int rl_moe_profile_enable(int on);
+int rl_moe_profile_read(float* stage_ms, int n);
+const char* rl_moe_profile_stage_name(int i);
+
+/* Kernel launches one rl_moe_prefill[_ws] call makes (for launch counting). */
+int rl_moe_launches_per_call(void);
+
+/* Thread-local message of the last failing call on this thread. */
+const char* rl_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RL_MOE_H */

@@ -1,0 +1,222 @@
+"""GPU parity of the CUDA path (through the C ABI) against the float64 oracle.
+
+Routing indices, offsets and the expert lists must match bit for bit; the
+routing weights within 1e-6; y within relative L2 5e-3 and
+max|diff| <= 2e-2 * rms(y_ref).  Small cases compare every output; the full
+workloads (launched exactly as bench.py launches them) compare sampled
+tokens, which the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+
+from bit_routed_expert_top_b200 import synth
+from oracle import moe_oracle as O
+from tests import helpers as Hh
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - CPU machine
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+from bit_routed_expert_top_b200 import api  # noqa: E402
+
+
+@pytest.fixture(autouse=True)
+def _tc_default():
+    api.debug_set_gemm("tc")
+    yield
+    api.debug_set_gemm("tc")
+
+
+def run_prefill(inp, ws=None):
+    wl = inp.wl
+    x, logits, blobs = Hh.to_device(inp)
+    y = torch.full((wl.T, wl.H), float("nan"), dtype=torch.float32, device="cuda")
+    if ws is None:
+        ws = api.alloc_workspace(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k)
+    api.rl_moe_prefill_ws(x, logits, blobs, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws)
+    bits = api.rl_moe_check_status(ws)
+    assert bits == 0, api.rl_last_error()
+    return y.cpu().numpy(), ws
+
+
+def run_route(logits_np, k):
+    T, E = logits_np.shape
+    logits = torch.from_numpy(np.ascontiguousarray(logits_np, dtype=np.float32)).cuda()
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    pl = torch.empty(max(T * k, 1), dtype=torch.int32, device="cuda")
+    pp = torch.empty(max(T * k, 1), dtype=torch.int32, device="cuda")
+    ws = api.alloc_workspace(2, T, 32, 32, E, k)
+    api.rl_moe_route(logits, T, E, k, idx, w, off, pl, pp, ws)
+    assert api.rl_moe_check_status(ws) == 0, api.rl_last_error()
+    return (idx.cpu().numpy(), w.cpu().numpy(), off.cpu().numpy(), pl.cpu().numpy()[:T * k],
+            pp.cpu().numpy()[:T * k])
+
+
+def check_route(logits_np, k):
+    idx, w, off, pl, pp = run_route(logits_np, k)
+    ridx, rp = O.route(logits_np, k)
+    roff, rpl, rpp = O.group(ridx, logits_np.shape[1])
+    np.testing.assert_array_equal(idx, ridx)
+    np.testing.assert_array_equal(off, roff)
+    np.testing.assert_array_equal(pl, rpl)
+    np.testing.assert_array_equal(pp, rpp)
+    np.testing.assert_allclose(w, rp, rtol=0, atol=Hh.P_ATOL)
+
+
+# ------------------------------------------------------------------ route ---
+
+@pytest.mark.parametrize("wi", range(len(synth.WORKLOADS)))
+def test_route_bit_exact_all_workloads(wi):
+    inp = synth.make_inputs(synth.WORKLOADS[wi])
+    check_route(inp.logits, inp.wl.k)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_route_ties_and_signed_zero(seed):
+    rng = np.random.default_rng(100 + seed)
+    vals = np.array([-1.0, -0.0, 0.0, 0.5, 1.0, 2.0], dtype=np.float32)
+    for (T, E, k) in [(37, 13, 3), (64, 512, 10), (5, 1024, 1024), (33, 16, 16)]:
+        logits = vals[rng.integers(0, len(vals), (T, E))]
+        check_route(logits, k)
+    # exact tie straddling the k / k+1 boundary
+    logits = np.zeros((3, 8), np.float32)
+    logits[:, [1, 6]] = 1.0
+    logits[1, 4] = -0.0
+    check_route(logits, 1)
+    check_route(logits, 3)
+
+
+def test_route_all_equal():
+    logits = np.full((70, 40), 0.5, np.float32)
+    idx, w, off, pl, pp = run_route(logits, 7)
+    assert (idx == np.arange(7)).all()
+    np.testing.assert_allclose(w, 1 / 7, atol=1e-7)
+
+
+# ------------------------------------------------------------ whole layer ---
+
+def full_oracle(inp):
+    return O.moe_prefill(inp.x_bits, inp.logits, Hh.oracle_blobs(inp), inp.wl.fmt, inp.wl.H,
+                         inp.wl.I, inp.wl.k, keep_intermediates=True)
+
+
+@pytest.mark.parametrize("wl", [
+    synth.WORKLOADS[0],                                             # tiny, Q2
+    synth.Workload("tiny_q1", 64, 256, 128, 16, 2, synth.FMT_Q1),
+    synth.Workload("ragged", 37, 96, 160, 9, 3, synth.FMT_Q2),     # T, H, I off every tile
+    synth.Workload("ragged_q1", 45, 352, 96, 7, 2, synth.FMT_Q1),
+    synth.Workload("t1", 1, 512, 256, 12, 4, synth.FMT_Q2),
+    synth.Workload("k_eq_e", 20, 256, 64, 6, 6, synth.FMT_Q1),
+    synth.Workload("k1", 50, 256, 128, 8, 1, synth.FMT_Q2),
+], ids=lambda w: w.name)
+def test_layer_small_every_output(wl):
+    inp = synth.make_inputs(wl, seed=sum(wl.name.encode()))
+    y, _ = run_prefill(inp)
+    ref = full_oracle(inp)
+    Hh.assert_y_close(y, ref["y"], wl.name)
+
+
+def test_layer_heavy_expert_many_n_tiles():
+    """One expert takes every token (n_e = T > one N tile), most experts
+    get no pair at all."""
+    wl = synth.Workload("heavy", 300, 256, 128, 24, 2, synth.FMT_Q2)
+    inp = synth.make_inputs(wl, seed=3)
+    inp.logits[:, 5] += 50.0
+    y, _ = run_prefill(inp)
+    ref = full_oracle(inp)
+    assert np.bincount(ref["idx"].ravel(), minlength=wl.E)[5] == wl.T
+    Hh.assert_y_close(y, ref["y"], "heavy")
+
+
+def test_layer_zero_down_is_zero():
+    wl = synth.Workload("zd", 40, 256, 128, 8, 2, synth.FMT_Q1)
+    inp = synth.make_inputs(wl, seed=9)
+    nb_gu = 2 * wl.I * 1 * 38
+    for e in range(wl.E):
+        for off in range(nb_gu, synth.expert_bytes(wl.fmt, wl.H, wl.I), 38):
+            inp.blobs[e, off:off + 2] = 0
+    y, _ = run_prefill(inp)
+    assert np.all(y == 0.0)
+
+
+def test_intermediates_h_and_o_tiny():
+    inp = synth.make_inputs(synth.WORKLOADS[0])
+    wl = inp.wl
+    y, ws = run_prefill(inp)
+    ref = full_oracle(inp)
+    n = api.rl_moe_workspace_bytes(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k)
+    P = wl.T * wl.k
+    raw = ws.cpu().numpy()
+    h_bytes = P * wl.I * 2
+    o_bytes = P * wl.H * 2
+    # h and o are the last two pieces of the workspace (256-byte aligned)
+    o_off = n - ((o_bytes + 255) // 256 * 256)
+    h_off = o_off - ((h_bytes + 255) // 256 * 256)
+    h = raw[h_off:h_off + h_bytes].view(np.float16).reshape(P, wl.I).astype(np.float64)
+    o = raw[o_off:o_off + o_bytes].view(np.float16).reshape(P, wl.H).astype(np.float64)
+    h = Hh.unpermute_k(h, wl.fmt)
+    rel_h = np.linalg.norm(h - ref["h"]) / np.linalg.norm(ref["h"])
+    rel_o = np.linalg.norm(o - ref["o"]) / np.linalg.norm(ref["o"])
+    assert rel_h < 2e-3, rel_h
+    assert rel_o < 2e-3, rel_o
+
+
+@pytest.mark.parametrize("wi", [1, 2, 3, 4])
+def test_full_workload_sampled_tokens(wi):
+    """Full-size workloads in bench.py's launch configuration; y of a sample
+    of tokens against the oracle, plus properties at every token."""
+    inp = synth.make_inputs(synth.WORKLOADS[wi])
+    wl = inp.wl
+    y, _ = run_prefill(inp)
+    assert np.all(np.isfinite(y))
+    rng = np.random.default_rng(wi)
+    toks = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 10)]))[:12]
+    _, _, yref = O.moe_prefill_tokens(inp.x_bits, inp.logits, Hh.oracle_blobs(inp), wl.fmt, wl.H,
+                                      wl.I, wl.k, toks)
+    Hh.assert_y_close(y[toks], yref, wl.name)
+
+
+def test_tc_matches_simt_stage_path():
+    """Tensor-core decode-GEMMs against the CUDA-core ones on the same inputs."""
+    wl = synth.Workload("x", 200, 512, 256, 32, 4, synth.FMT_Q2)
+    inp = synth.make_inputs(wl, seed=21)
+    y_tc, _ = run_prefill(inp)
+    api.debug_set_gemm("simt")
+    y_simt, _ = run_prefill(inp)
+    rel = np.linalg.norm(y_tc - y_simt) / np.linalg.norm(y_simt)
+    assert rel < 1e-3, rel
+
+
+def test_auto_workspace_entry_point_and_t0():
+    inp = synth.make_inputs(synth.WORKLOADS[0])
+    wl = inp.wl
+    x, logits, blobs = Hh.to_device(inp)
+    y = torch.empty((wl.T, wl.H), dtype=torch.float32, device="cuda")
+    api.rl_moe_prefill(x, logits, blobs, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y)
+    torch.cuda.synchronize()
+    ref = full_oracle(inp)
+    Hh.assert_y_close(y.cpu().numpy(), ref["y"], "auto-ws")
+    api.rl_moe_prefill(x, logits, blobs, wl.fmt, 0, wl.H, wl.I, wl.E, wl.k, y)
+
+
+def test_misaligned_blob_rejected():
+    inp = synth.make_inputs(synth.WORKLOADS[0])
+    wl = inp.wl
+    x, logits, blobs = Hh.to_device(inp)
+    flat = blobs.view(-1)
+    ptrs = [flat[e * inp.stride + (8 if e == 3 else 0):] for e in range(wl.E)]
+    y = torch.empty((wl.T, wl.H), dtype=torch.float32, device="cuda")
+    ws = api.alloc_workspace(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k)
+    with pytest.raises(api.RlMoeError, match="aligned"):
+        api.rl_moe_prefill_ws(x, logits, ptrs, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws)
+
+
+def test_repeat_calls_deterministic():
+    inp = synth.make_inputs(synth.WORKLOADS[2])
+    y1, ws = run_prefill(inp)
+    y2, _ = run_prefill(inp, ws)
+    np.testing.assert_array_equal(y1, y2)
