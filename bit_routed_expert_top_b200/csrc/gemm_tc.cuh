@@ -1,23 +1,631 @@
-// gemm_tc.cuh - tensor-core decode-GEMMs (placeholder: routes to the CUDA-core kernels).
+// gemm_tc.cuh - steps 3 and 4 on the sm_100a tensor cores: grouped
+// decode-GEMMs whose weights are decoded on the fly from Q1/Q2 blocks into
+// tensor memory and multiplied by tcgen05.mma.
+//
+// The Red Lite pages find the routed experts bound by decoding their weights
+// ("Red Lite dev75 - --kv f16, faster prompt ingestion", section 2: decoding
+// every 16-pair slice; whole-expert dequantization would write ~6 GB per
+// layer) and the gate/up kernel bound by instruction issue with a third of its
+// instructions spent on bit decoding ("Red Lite dev72 - bounded verify,
+// profiling", section 4, second profile).  Here the decode runs once per
+// (weight, unit of up to 128 pairs) on the CUDA cores and the products run on
+// the tensor cores, so the decode is the only per-weight integer work:
+//
+//   * weights are the A operand and live in TMEM (tcgen05.mma ... [a_tmem]):
+//     decoder threads write their row (= TMEM lane) with tcgen05.st, so the
+//     decoded tiles never round-trip through shared memory;
+//   * M = 128 weight rows, N = the unit's pairs rounded up to 16 (the pages'
+//     32-pair tiles lost because the partial tile wasted matrix work, dev72
+//     section 4; here the waste is at most 15 columns), K = 16 per MMA;
+//   * B = the unit's activation rows (x for gate/up, h for down) gathered
+//     into shared memory in the canonical no-swizzle K-major layout;
+//   * gate and up are two M tiles of one unit sharing B, so both run in one
+//     pass (two passes over the pairs lost on the pages, dev76 section 3),
+//     and the SwiGLU runs in the epilogue on the two TMEM accumulators.
+//
+// Warp roles (19 warps, one CTA per SM, persistent over the unit list):
+//   warp 0       TMEM allocation and the single MMA-issuing thread
+//   warp 1       raw weight blocks: one cp.async.bulk per (row, block)
+//   warp 2       B operand gather: cp.async 16-byte pieces
+//   warps 3..18  16 decoders (4 groups = 2 M tiles x 2 sub-block parities,
+//                one warp per TMEM lane quarter), then the epilogue
+// Every wait is bounded: on timeout the CTA raises RL_DEV_WAIT_TIMEOUT in
+// the status word and all roles leave their loops.
 #pragma once
+
 #include "common.cuh"
-#include "gemm_simt.cuh"
 
 namespace rl {
 namespace tc {
-constexpr int kNtGu = 128;
-constexpr int kNtDn = 128;
-constexpr int kMtDn = 2;
+
+constexpr int kNtGu = 128;       // max pairs per gate/up unit (N of the MMA)
+constexpr int kNtDn = 128;       // max pairs per down unit
+constexpr int kMtDn = 2;         // 128-row slabs per down unit
+constexpr int kMT = 2;           // M tiles per unit (gate+up, or two down slabs)
+constexpr int kNT = 128;         // accumulator columns per M tile
+constexpr int kRing = 8;         // A sub-block stages in TMEM
+constexpr int kRingCol = kMT * kNT;            // first ring column (256)
+constexpr int kSlotCols = 16;                  // 32 fp16 of K per lane
+constexpr int kRawStages = 3;
+constexpr int kBStages = 3;
+constexpr int kBK = 128;                       // K values per B stage
+constexpr int kBLbo = (kNT / 8) * 128;         // bytes between K core matrices (2048)
+constexpr int kBStageBytes = (kBK / 8) * kBLbo;  // 32 KB
+constexpr int kRows = kMT * 128;               // weight rows per unit
+constexpr int kWarps = 19;
+constexpr int kThreads = kWarps * 32;
+constexpr int kDecWarp0 = 3;
+constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+
+template <int FMT> struct Raw;
+template <> struct Raw<RL_FMT_Q2> { static constexpr int kPitch = 112; };  // >= 69+15, 16*odd
+template <> struct Raw<RL_FMT_Q1> { static constexpr int kPitch = 80; };   // >= 38+15, 16*odd
+
+template <int FMT>
+__host__ __device__ constexpr int raw_stage_bytes() { return kRows * Raw<FMT>::kPitch; }
+
+template <int FMT>
+__host__ __device__ constexpr int smem_bytes() {
+  return kRawStages * raw_stage_bytes<FMT>() + kBStages * kBStageBytes + 1024;
+}
+
+// ------------------------------------------------------------------ PTX ---
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// D[tmem] (+)= A[tmem] * B[smem], fp16 x fp16 -> fp32, cta_group::1.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_addr(bar))
+               : "memory");
+}
+
+// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B fp16
+// (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 in bits
+// 17-22, M >> 4 in bits 24-28.
+__device__ __forceinline__ uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Shared-memory matrix descriptor, no swizzle, K-major: start address,
+// leading byte offset (next 8-value core matrix along K), stride byte offset
+// (next group of 8 rows along N), all >> 4; version 1 in bits 46-47.
+__device__ __forceinline__ uint64_t sdesc_noswizzle(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+struct Shared {
+  uint64_t full_raw[kRawStages], empty_raw[kRawStages];
+  uint64_t full_b[kBStages], empty_b[kBStages];
+  uint64_t full_a[kRing], empty_a[kRing];
+  uint64_t acc_full, acc_empty, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int toks[kNT];
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared* sh, unsigned* status) {
+  const uint32_t addr = smem_addr(bar);
+  long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if ((it & 31u) == 31u) {
+      if (*(volatile int*)&sh->abort_flag) return false;
+      const long long now = clock64();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitCycles) {
+        *(volatile int*)&sh->abort_flag = 1;
+        atomicOr(status, RL_DEV_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------ decoding ---
+// fp16 LUT of one sub-block.  Q2: bytes 2u, 2u+1 of (lo, hi) hold
+// fp16(d(2s+1)(2u-3)), u = 0..3; Q1: bytes 2b, 2b+1 of lo hold
+// fp16(d(2s+1)((2b-1)+delta)).  d(2s+1) and its product with the code are
+// exact in fp32, so each weight is rounded exactly once.
+template <int FMT>
+__device__ __forceinline__ void make_lut(float dd, uint32_t S, uint32_t flags, int i, uint32_t& lo,
+                                         uint32_t& hi) {
+  const float m = dd * (float)(2u * ((S >> (3 * i)) & 7u) + 1u);
+  if constexpr (FMT == RL_FMT_Q2) {
+    const __half2 p = __floats2half2_rn(m, 3.0f * m);          // u=2 (low), u=3 (high)
+    hi = *reinterpret_cast<const uint32_t*>(&p);
+    lo = __byte_perm(hi, 0u, 0x1032) ^ 0x80008000u;            // u=0: -3m, u=1: -m
+  } else {
+    const float delta = ((flags >> i) & 1u) ? 0.125f : -0.125f;
+    const __half2 p = __floats2half2_rn(m * (delta - 1.0f), m * (delta + 1.0f));
+    lo = *reinterpret_cast<const uint32_t*>(&p);
+    hi = lo;
+  }
+}
+
+// One 32-bit code word -> fp16x2 words out[0 .. G/2).  Word 2k+h holds the
+// values (k + 2h*P, k + (2h+1)*P) of the group, P = codes per byte, i.e.
+// position i holds value (i >> 2) + P*(i & 3).
+template <int FMT>
+__device__ __forceinline__ void decode_word(uint32_t c, uint32_t lo, uint32_t hi, uint32_t* out) {
+  constexpr int P = Fmt<FMT>::kPerByte;
+  constexpr uint32_t mask = FMT == RL_FMT_Q2 ? 0x03030303u : 0x01010101u;
+#pragma unroll
+  for (int k = 0; k < P; ++k) {
+    const uint32_t v = (c >> (Fmt<FMT>::kBits * k)) & mask;
+    const uint32_t sel = v * 0x22u + 0x10101010u;
+    out[2 * k] = __byte_perm(lo, hi, sel);
+    out[2 * k + 1] = __byte_perm(lo, hi, sel >> 16);
+  }
+}
+
+// 8 bytes starting at byte offset o of a shared-memory row region (o may be
+// unaligned; the region is 16-byte aligned and padded).
+__device__ __forceinline__ void load8_unaligned(const uint8_t* region, int o, uint32_t& w0, uint32_t& w1) {
+  const int u = o & ~7;
+  const uint2 a = *reinterpret_cast<const uint2*>(region + u);
+  const uint2 b = *reinterpret_cast<const uint2*>(region + u + 8);
+  const int sh = o & 7;
+  const bool hi4 = sh >= 4;
+  const uint32_t x0 = hi4 ? a.y : a.x;
+  const uint32_t x1 = hi4 ? b.x : a.y;
+  const uint32_t x2 = hi4 ? b.y : b.x;
+  const uint32_t s = (uint32_t)(sh & 3) * 8u;
+  w0 = __funnelshift_r(x0, x1, s);
+  w1 = __funnelshift_r(x1, x2, s);
+}
+
+// ------------------------------------------------------------- kernel ---
+// GATEUP: unit {expert, slab, n0, cnt}: tile 0 = gate rows 128*slab + r,
+//         tile 1 = up rows 128*slab + r; K = H; B = x16 rows of the pairs'
+//         tokens; epilogue h = silu(g)*u -> h16 (grouped order, K-permuted).
+// DOWN:   unit {expert, group, n0, cnt}: tile t = down rows 128*(2*group+t)+r;
+//         K = I; B = h16 rows n0..n0+cnt; epilogue o16[pair][row] = fp16(acc).
+template <int FMT, bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  uint8_t* raw_base = smem;
+  uint8_t* b_base = raw_base + kRawStages * raw_stage_bytes<FMT>();
+  Shared* sh = reinterpret_cast<Shared*>(b_base + kBStages * kBStageBytes);
+
+  constexpr int BB = Fmt<FMT>::kBytes;
+  constexpr int PITCH = Raw<FMT>::kPitch;
+  const int n_units = w.counters[GATEUP ? 0 : 1];
+  if ((int)blockIdx.x >= n_units) return;
+  const int4* units = GATEUP ? w.units_gu : w.units_dn;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = GATEUP ? d.H : d.I;
+  const int nsub = K / kSubVals;
+  const int nblk = GATEUP ? d.nbH : d.nbI;
+  const int nbchunk = (K + kBK - 1) / kBK;
+  const size_t rowbytes = (size_t)nblk * BB;
+  const size_t gu_rowbytes = (size_t)d.nbH * BB;
+  const int rows_total = GATEUP ? d.I : d.H;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRawStages; ++s) {
+      mbar_init(&sh->full_raw[s], 32);
+      mbar_init(&sh->empty_raw[s], 16);
+    }
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&sh->full_b[s], 1);
+      mbar_init(&sh->empty_b[s], 1);
+    }
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&sh->full_a[s], kMT * 4);
+      mbar_init(&sh->empty_a[s], 1);
+    }
+    mbar_init(&sh->acc_full, 1);
+    mbar_init(&sh->acc_empty, 16);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(&sh->tmem_base)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ MMA ---
+    if (lane == 0) {
+      uint32_t ring_it = 0, b_it = 0, u_it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_it) {
+        const int4 un = units[u];
+        const int npad = max(16, (un.w + 15) & ~15);
+        const uint32_t idesc = idesc_f16(128, npad);
+        if (u_it > 0) ok = wait_bar(&sh->acc_empty, (u_it - 1) & 1, sh, w.status);
+        tc_fence_after();
+        for (int sb = 0; sb < nsub && ok; ++sb) {
+          const uint32_t bi = b_it + sb / (kBK / kSubVals);
+          const int bs = bi % kBStages;
+          if (sb % (kBK / kSubVals) == 0) {
+            ok = wait_bar(&sh->full_b[bs], (bi / kBStages) & 1, sh, w.status);
+            if (!ok) break;
+          }
+          const uint32_t ai = ring_it + sb;
+          const int as = ai % kRing;
+          ok = wait_bar(&sh->full_a[as], (ai / kRing) & 1, sh, w.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t bstage = smem_addr(b_base + bs * kBStageBytes);
+          const int kin = (sb % (kBK / kSubVals)) * kSubVals;   // K offset inside the B stage
+#pragma unroll
+          for (int t = 0; t < kMT; ++t) {
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const uint32_t a_tm = tmem + kRingCol + as * (kMT * kSlotCols) + t * kSlotCols + kk * 8;
+              const uint64_t bd = sdesc_noswizzle(bstage + ((kin + kk * 16) / 8) * kBLbo, kBLbo, 128);
+              mma_ts(tmem + t * kNT, a_tm, bd, idesc, (sb | kk) != 0);
+            }
+          }
+          mma_commit(&sh->empty_a[as]);
+          if (sb % (kBK / kSubVals) == (kBK / kSubVals) - 1 || sb == nsub - 1) mma_commit(&sh->empty_b[bs]);
+        }
+        if (ok) mma_commit(&sh->acc_full);
+        ring_it += nsub;
+        b_it += nbchunk;
+      }
+      // drain: every MMA issued by this thread has completed before teardown
+      mma_commit(&sh->drain);
+      wait_bar(&sh->drain, 0, sh, w.status);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------- raw weight blocks -------
+    uint32_t raw_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int4 un = units[u];
+      const uint8_t* blob = tab.p[un.x];
+      for (int kb = 0; kb < nblk && ok; ++kb, ++raw_it) {
+        const int s = raw_it % kRawStages;
+        ok = __all_sync(0xffffffffu, wait_bar(&sh->empty_raw[s], ((raw_it / kRawStages) & 1) ^ 1, sh, w.status));
+        if (!ok) break;
+        uint8_t* stage = raw_base + s * raw_stage_bytes<FMT>();
+        // lane handles rows rho = lane + 32*j
+        uint32_t bytes = 0;
+        const uint8_t* src[kRows / 32];
+        uint32_t len[kRows / 32];
+#pragma unroll
+        for (int j = 0; j < kRows / 32; ++j) {
+          const int rho = lane + 32 * j;
+          const int t = rho >> 7, r = rho & 127;
+          int R;
+          const uint8_t* mat;
+          if (GATEUP) {
+            R = un.y * 128 + r;
+            mat = blob + (size_t)t * d.I * gu_rowbytes;
+          } else {
+            R = (un.y * kMT + t) * 128 + r;
+            mat = blob + (size_t)2 * d.I * gu_rowbytes;
+          }
+          len[j] = 0;
+          src[j] = nullptr;
+          if (R < rows_total) {
+            const uint8_t* b0 = mat + (size_t)R * rowbytes + (size_t)kb * BB;
+            const uintptr_t a0 = reinterpret_cast<uintptr_t>(b0) & ~(uintptr_t)15;
+            const uintptr_t a1 = (reinterpret_cast<uintptr_t>(b0) + BB + 15) & ~(uintptr_t)15;
+            src[j] = reinterpret_cast<const uint8_t*>(a0);
+            len[j] = (uint32_t)(a1 - a0);
+            bytes += len[j];
+          }
+        }
+        mbar_arrive_expect_tx(&sh->full_raw[s], bytes);
+#pragma unroll
+        for (int j = 0; j < kRows / 32; ++j)
+          if (len[j]) bulk_g2s(stage + (lane + 32 * j) * PITCH, src[j], len[j], &sh->full_raw[s]);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------- B operand gather --------
+    uint32_t b_it = 0;
+    bool ok = true;
+    int pending = -1;                      // stage whose copies are in flight
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int4 un = units[u];
+      const int cnt = un.w, n0 = un.z;
+      const int npad = max(16, (cnt + 15) & ~15);
+      // the previous unit's last stage must land before toks is rewritten
+      if (pending >= 0) {
+        cp_async_wait<0>();
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->full_b[pending]);
+        pending = -1;
+      }
+      for (int n = lane; n < cnt; n += 32)
+        sh->toks[n] = GATEUP ? w.pair_list[n0 + n] / d.k : n0 + n;
+      __syncwarp();
+      const __half* src_base = GATEUP ? w.x16 : w.h16;
+      for (int kc = 0; kc < nbchunk && ok; ++kc, ++b_it) {
+        const int s = b_it % kBStages;
+        ok = __all_sync(0xffffffffu, wait_bar(&sh->empty_b[s], ((b_it / kBStages) & 1) ^ 1, sh, w.status));
+        if (!ok) break;
+        uint8_t* stage = b_base + s * kBStageBytes;
+        const int kbase = kc * kBK;
+        const int kvalid = min(kBK, K - kbase);
+        for (int g8 = 0; g8 < npad / 8; ++g8) {
+          const int n = g8 * 8 + (lane & 7);
+          const int tok = n < cnt ? sh->toks[n] : 0;
+          const __half* rowp = src_base + (size_t)tok * K + kbase;
+#pragma unroll
+          for (int quad = 0; quad < kBK / 32; ++quad) {
+            const int c = quad * 4 + (lane >> 3);          // 8-value chunk inside the stage
+            if (n < cnt && c * 8 < kvalid)
+              cp_async16(stage + c * kBLbo + g8 * 128 + (lane & 7) * 16, rowp + c * 8);
+          }
+        }
+        cp_async_commit();
+        if (pending >= 0) {
+          cp_async_wait<1>();
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->full_b[pending]);
+        }
+        pending = s;
+      }
+    }
+    if (pending >= 0) {
+      cp_async_wait<0>();
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->full_b[pending]);
+    }
+  } else {
+    // ------------------------------------------- decoders + epilogue -----
+    const int dw = warp - kDecWarp0;          // 0..15
+    const int grp = dw >> 2;                  // 0..3
+    const int tile = grp & 1, parity = grp >> 1;
+    const int q = warp & 3;                   // TMEM lane quarter
+    const int r = q * 32 + lane;              // lane = row inside the tile
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    uint32_t raw_it = 0, ring_it = 0, u_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_it) {
+      const int4 un = units[u];
+      const uint8_t* blob = tab.p[un.x];
+      const int rho = tile * 128 + r;
+      int R;
+      const uint8_t* mat;
+      if (GATEUP) {
+        R = un.y * 128 + r;
+        mat = blob + (size_t)tile * d.I * gu_rowbytes;
+      } else {
+        R = (un.y * kMT + tile) * 128 + r;
+        mat = blob + (size_t)2 * d.I * gu_rowbytes;
+      }
+      const bool valid = R < rows_total;
+      const uint8_t* rowg = mat + (size_t)(valid ? R : 0) * rowbytes;
+      for (int kb = 0; kb < nblk && ok; ++kb) {
+        const uint32_t ri = raw_it + kb;
+        const int rs = ri % kRawStages;
+        ok = __all_sync(0xffffffffu, wait_bar(&sh->full_raw[rs], (ri / kRawStages) & 1, sh, w.status));
+        if (!ok) break;
+        const uint8_t* region = raw_base + rs * raw_stage_bytes<FMT>() + rho * PITCH;
+        const int off = (int)(reinterpret_cast<uintptr_t>(rowg + (size_t)kb * BB) & 15);
+        uint32_t h0, h1;
+        load8_unaligned(region, off, h0, h1);
+        const float dd = half_bits_to_float(h0 & 0xffffu);
+        const uint32_t S = (h0 >> 16) | ((h1 & 0xffu) << 16);
+        const uint32_t flags = (h1 >> 8) & 0xffu;
+        for (int i = parity; i < 8 && ok; i += 2) {
+          const int sb = kb * 8 + i;
+          if (sb >= nsub) break;
+          uint32_t words[16];
+          if (valid) {
+            uint32_t lo, hi;
+            make_lut<FMT>(dd, S, flags, i, lo, hi);
+            if constexpr (FMT == RL_FMT_Q2) {
+              uint32_t c0, c1;
+              load8_unaligned(region, off + 5 + 8 * i, c0, c1);
+              decode_word<FMT>(c0, lo, hi, words);
+              decode_word<FMT>(c1, lo, hi, words + 8);
+            } else {
+              uint32_t c0, c1;
+              load8_unaligned(region, off + 6 + 4 * i, c0, c1);
+              decode_word<FMT>(c0, lo, hi, words);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) words[j] = 0u;
+          }
+          const uint32_t ai = ring_it + sb;
+          const int as = ai % kRing;
+          ok = __all_sync(0xffffffffu, wait_bar(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status));
+          if (!ok) break;
+          tc_fence_after();
+          tmem_st16(tmem + lane_addr + kRingCol + as * (kMT * kSlotCols) + tile * kSlotCols, words);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->full_a[as]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->empty_raw[rs]);
+      }
+      raw_it += nblk;
+      ring_it += nsub;
+      if (!ok) break;
+
+      // epilogue
+      ok = __all_sync(0xffffffffu, wait_bar(&sh->acc_full, u_it & 1, sh, w.status));
+      if (!ok) break;
+      tc_fence_after();
+      const int cnt = un.w, n0 = un.z;
+      const int npad = max(16, (cnt + 15) & ~15);
+      for (int cc = grp; cc < npad / 16; cc += 4) {
+        uint32_t a0[16], a1[16];
+        tmem_ld16(tmem + lane_addr + 0 * kNT + cc * 16, a0);
+        tmem_ld16(tmem + lane_addr + 1 * kNT + cc * 16, a1);
+        tmem_wait_ld();
+        if (GATEUP) {
+          const int rr = un.y * 128 + r;
+          if (rr < d.I) {
+            const int pos = perm_pos_k<FMT>(rr);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = cc * 16 + j;
+              if (n < cnt) {
+                const float g = __uint_as_float(a0[j]);
+                const float uu = __uint_as_float(a1[j]);
+                const float hv = g / (1.0f + __expf(-g)) * uu;
+                w.h16[(size_t)(n0 + n) * d.I + pos] = __float2half_rn(hv);
+              }
+            }
+          }
+        } else {
+          const int r0 = (un.y * kMT) * 128 + r;
+          const int r1 = r0 + 128;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = cc * 16 + j;
+            if (n < cnt) {
+              const int pid = __ldg(w.pair_list + n0 + n);
+              if (r0 < d.H) w.o16[(size_t)pid * d.H + r0] = __float2half_rn(__uint_as_float(a0[j]));
+              if (r1 < d.H) w.o16[(size_t)pid * d.H + r1] = __float2half_rn(__uint_as_float(a1[j]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+  }
+}
+
+inline int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int FMT, bool GATEUP>
+int launch(const Dims& d, const Work& w, const ExpertTable& tab, cudaStream_t s) {
+  static bool configured = false;
+  constexpr int smem = smem_bytes<FMT>();
+  if (!configured) {
+    const cudaError_t e = cudaFuncSetAttribute(decode_gemm_kernel<FMT, GATEUP>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return RL_ERR_CUDA;
+    configured = true;
+  }
+  const int maxu = GATEUP ? d.max_units_gu : d.max_units_dn;
+  const int grid = maxu < num_sms() ? maxu : num_sms();
+  decode_gemm_kernel<FMT, GATEUP><<<grid, kThreads, smem, s>>>(d, w, tab);
+  return RL_OK;
+}
 
 template <int FMT>
 int launch_gateup(const Dims& d, const Work& w, const ExpertTable& tab, cudaStream_t s) {
-  gateup_simt_kernel<FMT><<<d.max_units_gu, 256, 0, s>>>(d, w, tab);
-  return RL_OK;
+  return launch<FMT, true>(d, w, tab, s);
 }
 template <int FMT>
 int launch_down(const Dims& d, const Work& w, const ExpertTable& tab, cudaStream_t s) {
-  down_simt_kernel<FMT><<<d.max_units_dn, 256, 0, s>>>(d, w, tab);
-  return RL_OK;
+  return launch<FMT, false>(d, w, tab, s);
 }
+
 }  // namespace tc
 }  // namespace rl
