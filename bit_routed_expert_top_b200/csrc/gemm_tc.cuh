@@ -8,7 +8,7 @@
 // layer) and the gate/up kernel bound by instruction issue with a third of its
 // instructions spent on bit decoding ("Red Lite dev72 - bounded verify,
 // profiling", section 4, second profile).  Here the decode runs once per
-// (weight, unit of up to 128 pairs) on the CUDA cores and the products run on
+// (weight, unit of up to 64 pairs) on the CUDA cores and the products run on
 // the tensor cores, so the decode is the only per-weight integer work:
 //
 //   * weights are the A operand and live in TMEM (tcgen05.mma ... [a_tmem]):
@@ -23,12 +23,15 @@
 //     pass (two passes over the pairs lost on the pages, dev76 section 3),
 //     and the SwiGLU runs in the epilogue on the two TMEM accumulators.
 //
-// Warp roles (19 warps, one CTA per SM, persistent over the unit list):
+// Warp roles (22 warps, one CTA per SM, persistent over the unit list):
 //   warp 0       TMEM allocation and the single MMA-issuing thread
-//   warp 1       raw weight blocks: one cp.async.bulk per (row, block)
-//   warp 2       B operand gather: cp.async 16-byte pieces
-//   warps 3..18  16 decoders (4 groups = 2 M tiles x 2 sub-block parities,
-//                one warp per TMEM lane quarter), then the epilogue
+//   warp 1       B operand gather (16-byte cp.async into the K-major layout)
+//   warps 2..5   epilogue (one per TMEM lane quarter), double-buffered
+//                accumulators so it overlaps the next unit's MMAs
+//   warps 6..21  16 decoders: 4 groups = 2 M tiles x 2 sub-block parities,
+//                one warp per lane quarter.  The warps of one parity also
+//                fetch the raw blocks of every other K block for their rows
+//                (16-byte cp.async, completion counted on an mbarrier).
 // Every wait is bounded: on timeout the CTA raises RL_DEV_WAIT_TIMEOUT in
 // the status word and all roles leave their loops.
 #pragma once
@@ -38,28 +41,34 @@
 namespace rl {
 namespace tc {
 
-constexpr int kNtGu = 128;       // max pairs per gate/up unit (N of the MMA)
-constexpr int kNtDn = 128;       // max pairs per down unit
+constexpr int kNT = 64;          // max pairs per unit = accumulator columns per tile
+constexpr int kNtGu = kNT;       // gate/up unit size in pairs
+constexpr int kNtDn = kNT;       // down unit size in pairs
 constexpr int kMtDn = 2;         // 128-row slabs per down unit
 constexpr int kMT = 2;           // M tiles per unit (gate+up, or two down slabs)
-constexpr int kNT = 128;         // accumulator columns per M tile
+constexpr int kAccBufs = 2;      // accumulator buffers (epilogue overlap)
 constexpr int kRing = 8;         // A sub-block stages in TMEM
-constexpr int kRingCol = kMT * kNT;            // first ring column (256)
-constexpr int kSlotCols = 16;                  // 32 fp16 of K per lane
-constexpr int kRawStages = 3;
-constexpr int kBStages = 3;
-constexpr int kBK = 128;                       // K values per B stage
-constexpr int kBLbo = (kNT / 8) * 128;         // bytes between K core matrices (2048)
-constexpr int kBStageBytes = (kBK / 8) * kBLbo;  // 32 KB
-constexpr int kRows = kMT * 128;               // weight rows per unit
-constexpr int kWarps = 19;
+constexpr int kRingCol = kAccBufs * kMT * kNT;  // first ring column (256)
+constexpr int kSlotCols = 16;                   // 32 fp16 of K per lane
+constexpr int kRawStages = 4;
+constexpr int kRawAhead = 2;                    // raw blocks fetched ahead
+constexpr int kBStages = 4;
+constexpr int kBK = 128;                        // K values per B stage
+constexpr int kBLbo = (kNT / 8) * 128;          // bytes between K core matrices (1024)
+constexpr int kBStageBytes = (kBK / 8) * kBLbo; // 16 KB
+constexpr int kRows = kMT * 128;                // weight rows per unit
+constexpr int kEpiWarp0 = 2;
+constexpr int kDecWarp0 = 6;
+constexpr int kWarps = 22;
 constexpr int kThreads = kWarps * 32;
-constexpr int kDecWarp0 = 3;
-constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+constexpr long long kWaitCycles = 4000000000LL; // ~2 s at 2 GHz
+static_assert(kRingCol + kRing * kMT * kSlotCols <= 512, "TMEM columns");
 
 template <int FMT> struct Raw;
-template <> struct Raw<RL_FMT_Q2> { static constexpr int kPitch = 112; };  // >= 69+15, 16*odd
-template <> struct Raw<RL_FMT_Q1> { static constexpr int kPitch = 80; };   // >= 38+15, 16*odd
+// row region: the 16-byte chunks that hold one block (<= 69+15 / 38+15 bytes),
+// pitch an odd number of 16-byte chunks
+template <> struct Raw<RL_FMT_Q2> { static constexpr int kPitch = 112; static constexpr int kChunks = 6; };
+template <> struct Raw<RL_FMT_Q1> { static constexpr int kPitch = 80; static constexpr int kChunks = 4; };
 
 template <int FMT>
 __host__ __device__ constexpr int raw_stage_bytes() { return kRows * Raw<FMT>::kPitch; }
@@ -174,7 +183,7 @@ struct Shared {
   uint64_t full_raw[kRawStages], empty_raw[kRawStages];
   uint64_t full_b[kBStages], empty_b[kBStages];
   uint64_t full_a[kRing], empty_a[kRing];
-  uint64_t acc_full, acc_empty, drain;
+  uint64_t acc_full[kAccBufs], acc_empty[kAccBufs], drain;
   uint32_t tmem_base;
   int abort_flag;
   int toks[kNT];
@@ -197,6 +206,13 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared*
       }
     }
   }
+}
+// Warp-uniform variant: every lane waits, the result is agreed with a vote.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, Shared* sh, unsigned* status) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, sh, status));
+}
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 // ------------------------------------------------------------ decoding ---
@@ -252,26 +268,41 @@ __device__ __forceinline__ void load8_unaligned(const uint8_t* region, int o, ui
   w1 = __funnelshift_r(x1, x2, s);
 }
 
-// ------------------------------------------------------------- kernel ---
-// GATEUP: unit {expert, slab, n0, cnt}: tile 0 = gate rows 128*slab + r,
-//         tile 1 = up rows 128*slab + r; K = H; B = x16 rows of the pairs'
-//         tokens; epilogue h = silu(g)*u -> h16 (grouped order, K-permuted).
-// DOWN:   unit {expert, group, n0, cnt}: tile t = down rows 128*(2*group+t)+r;
-//         K = I; B = h16 rows n0..n0+cnt; epilogue o16[pair][row] = fp16(acc).
+// Rows of a unit.  GATEUP: unit {expert, slab, n0, cnt}: tile 0 = gate rows
+// 128*slab + r, tile 1 = up rows 128*slab + r, K = H.  DOWN: unit
+// {expert, group, n0, cnt}: tile t = down rows 128*(2*group+t) + r, K = I.
+template <bool GATEUP>
+__device__ __forceinline__ const uint8_t* tile_row(const Dims& d, const uint8_t* blob, int slab_or_group,
+                                                   int t, int r, size_t gu_rowbytes, size_t rowbytes,
+                                                   int* R_out) {
+  int R;
+  const uint8_t* mat;
+  if (GATEUP) {
+    R = slab_or_group * 128 + r;
+    mat = blob + (size_t)t * d.I * gu_rowbytes;
+  } else {
+    R = (slab_or_group * kMT + t) * 128 + r;
+    mat = blob + (size_t)2 * d.I * gu_rowbytes;
+  }
+  *R_out = R;
+  return mat + (size_t)R * rowbytes;
+}
+
 template <int FMT, bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = smem_raw;
-  uint8_t* raw_base = smem;
+  uint8_t* raw_base = smem_raw;
   uint8_t* b_base = raw_base + kRawStages * raw_stage_bytes<FMT>();
   Shared* sh = reinterpret_cast<Shared*>(b_base + kBStages * kBStageBytes);
 
   constexpr int BB = Fmt<FMT>::kBytes;
   constexpr int PITCH = Raw<FMT>::kPitch;
+  constexpr int CHUNKS = Raw<FMT>::kChunks;
   const int n_units = w.counters[GATEUP ? 0 : 1];
   if ((int)blockIdx.x >= n_units) return;
   const int4* units = GATEUP ? w.units_gu : w.units_dn;
+  const int my_units = (n_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = GATEUP ? d.H : d.I;
@@ -284,8 +315,8 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRawStages; ++s) {
-      mbar_init(&sh->full_raw[s], 32);
-      mbar_init(&sh->empty_raw[s], 16);
+      mbar_init(&sh->full_raw[s], 8 * 32);   // 8 fetching warps x 32 lanes (cp.async arrivals)
+      mbar_init(&sh->empty_raw[s], 16);      // all decoder warps
     }
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(&sh->full_b[s], 1);
@@ -295,8 +326,10 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
       mbar_init(&sh->full_a[s], kMT * 4);
       mbar_init(&sh->empty_a[s], 1);
     }
-    mbar_init(&sh->acc_full, 1);
-    mbar_init(&sh->acc_empty, 16);
+    for (int b = 0; b < kAccBufs; ++b) {
+      mbar_init(&sh->acc_full[b], 1);
+      mbar_init(&sh->acc_empty[b], 4);
+    }
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -316,14 +349,16 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
   if (warp == 0) {
     // ------------------------------------------------------------ MMA ---
     if (lane == 0) {
-      uint32_t ring_it = 0, b_it = 0, u_it = 0;
+      uint32_t ring_it = 0, b_it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_it) {
-        const int4 un = units[u];
+      for (int ui = 0; ui < my_units && ok; ++ui) {
+        const int4 un = units[blockIdx.x + ui * gridDim.x];
         const int npad = max(16, (un.w + 15) & ~15);
         const uint32_t idesc = idesc_f16(128, npad);
-        if (u_it > 0) ok = wait_bar(&sh->acc_empty, (u_it - 1) & 1, sh, w.status);
+        const int buf = ui & 1;
+        if (ui >= kAccBufs) ok = wait_bar(&sh->acc_empty[buf], ((ui / kAccBufs) - 1) & 1, sh, w.status);
         tc_fence_after();
+        const uint32_t acc0 = tmem + buf * (kMT * kNT);
         for (int sb = 0; sb < nsub && ok; ++sb) {
           const uint32_t bi = b_it + sb / (kBK / kSubVals);
           const int bs = bi % kBStages;
@@ -344,13 +379,13 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
             for (int kk = 0; kk < 2; ++kk) {
               const uint32_t a_tm = tmem + kRingCol + as * (kMT * kSlotCols) + t * kSlotCols + kk * 8;
               const uint64_t bd = sdesc_noswizzle(bstage + ((kin + kk * 16) / 8) * kBLbo, kBLbo, 128);
-              mma_ts(tmem + t * kNT, a_tm, bd, idesc, (sb | kk) != 0);
+              mma_ts(acc0 + t * kNT, a_tm, bd, idesc, (sb | kk) != 0);
             }
           }
           mma_commit(&sh->empty_a[as]);
           if (sb % (kBK / kSubVals) == (kBK / kSubVals) - 1 || sb == nsub - 1) mma_commit(&sh->empty_b[bs]);
         }
-        if (ok) mma_commit(&sh->acc_full);
+        if (ok) mma_commit(&sh->acc_full[buf]);
         ring_it += nsub;
         b_it += nbchunk;
       }
@@ -360,58 +395,12 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------- raw weight blocks -------
-    uint32_t raw_it = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int4 un = units[u];
-      const uint8_t* blob = tab.p[un.x];
-      for (int kb = 0; kb < nblk && ok; ++kb, ++raw_it) {
-        const int s = raw_it % kRawStages;
-        ok = __all_sync(0xffffffffu, wait_bar(&sh->empty_raw[s], ((raw_it / kRawStages) & 1) ^ 1, sh, w.status));
-        if (!ok) break;
-        uint8_t* stage = raw_base + s * raw_stage_bytes<FMT>();
-        // lane handles rows rho = lane + 32*j
-        uint32_t bytes = 0;
-        const uint8_t* src[kRows / 32];
-        uint32_t len[kRows / 32];
-#pragma unroll
-        for (int j = 0; j < kRows / 32; ++j) {
-          const int rho = lane + 32 * j;
-          const int t = rho >> 7, r = rho & 127;
-          int R;
-          const uint8_t* mat;
-          if (GATEUP) {
-            R = un.y * 128 + r;
-            mat = blob + (size_t)t * d.I * gu_rowbytes;
-          } else {
-            R = (un.y * kMT + t) * 128 + r;
-            mat = blob + (size_t)2 * d.I * gu_rowbytes;
-          }
-          len[j] = 0;
-          src[j] = nullptr;
-          if (R < rows_total) {
-            const uint8_t* b0 = mat + (size_t)R * rowbytes + (size_t)kb * BB;
-            const uintptr_t a0 = reinterpret_cast<uintptr_t>(b0) & ~(uintptr_t)15;
-            const uintptr_t a1 = (reinterpret_cast<uintptr_t>(b0) + BB + 15) & ~(uintptr_t)15;
-            src[j] = reinterpret_cast<const uint8_t*>(a0);
-            len[j] = (uint32_t)(a1 - a0);
-            bytes += len[j];
-          }
-        }
-        mbar_arrive_expect_tx(&sh->full_raw[s], bytes);
-#pragma unroll
-        for (int j = 0; j < kRows / 32; ++j)
-          if (len[j]) bulk_g2s(stage + (lane + 32 * j) * PITCH, src[j], len[j], &sh->full_raw[s]);
-      }
-    }
-  } else if (warp == 2) {
     // ------------------------------------------- B operand gather --------
     uint32_t b_it = 0;
     bool ok = true;
     int pending = -1;                      // stage whose copies are in flight
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int4 un = units[u];
+    for (int ui = 0; ui < my_units && ok; ++ui) {
+      const int4 un = units[blockIdx.x + ui * gridDim.x];
       const int cnt = un.w, n0 = un.z;
       const int npad = max(16, (cnt + 15) & ~15);
       // the previous unit's last stage must land before toks is rewritten
@@ -428,7 +417,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
       const __half* src_base = GATEUP ? w.x16 : w.h16;
       for (int kc = 0; kc < nbchunk && ok; ++kc, ++b_it) {
         const int s = b_it % kBStages;
-        ok = __all_sync(0xffffffffu, wait_bar(&sh->empty_b[s], ((b_it / kBStages) & 1) ^ 1, sh, w.status));
+        ok = wait_bar_warp(&sh->empty_b[s], ((b_it / kBStages) & 1) ^ 1, sh, w.status);
         if (!ok) break;
         uint8_t* stage = b_base + s * kBStageBytes;
         const int kbase = kc * kBK;
@@ -460,105 +449,34 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->full_b[pending]);
     }
-  } else {
-    // ------------------------------------------- decoders + epilogue -----
-    const int dw = warp - kDecWarp0;          // 0..15
-    const int grp = dw >> 2;                  // 0..3
-    const int tile = grp & 1, parity = grp >> 1;
-    const int q = warp & 3;                   // TMEM lane quarter
-    const int r = q * 32 + lane;              // lane = row inside the tile
+  } else if (warp < kDecWarp0) {
+    // ------------------------------------------------------ epilogue -----
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-    uint32_t raw_it = 0, ring_it = 0, u_it = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++u_it) {
-      const int4 un = units[u];
-      const uint8_t* blob = tab.p[un.x];
-      const int rho = tile * 128 + r;
-      int R;
-      const uint8_t* mat;
-      if (GATEUP) {
-        R = un.y * 128 + r;
-        mat = blob + (size_t)tile * d.I * gu_rowbytes;
-      } else {
-        R = (un.y * kMT + tile) * 128 + r;
-        mat = blob + (size_t)2 * d.I * gu_rowbytes;
-      }
-      const bool valid = R < rows_total;
-      const uint8_t* rowg = mat + (size_t)(valid ? R : 0) * rowbytes;
-      for (int kb = 0; kb < nblk && ok; ++kb) {
-        const uint32_t ri = raw_it + kb;
-        const int rs = ri % kRawStages;
-        ok = __all_sync(0xffffffffu, wait_bar(&sh->full_raw[rs], (ri / kRawStages) & 1, sh, w.status));
-        if (!ok) break;
-        const uint8_t* region = raw_base + rs * raw_stage_bytes<FMT>() + rho * PITCH;
-        const int off = (int)(reinterpret_cast<uintptr_t>(rowg + (size_t)kb * BB) & 15);
-        uint32_t h0, h1;
-        load8_unaligned(region, off, h0, h1);
-        const float dd = half_bits_to_float(h0 & 0xffffu);
-        const uint32_t S = (h0 >> 16) | ((h1 & 0xffu) << 16);
-        const uint32_t flags = (h1 >> 8) & 0xffu;
-        for (int i = parity; i < 8 && ok; i += 2) {
-          const int sb = kb * 8 + i;
-          if (sb >= nsub) break;
-          uint32_t words[16];
-          if (valid) {
-            uint32_t lo, hi;
-            make_lut<FMT>(dd, S, flags, i, lo, hi);
-            if constexpr (FMT == RL_FMT_Q2) {
-              uint32_t c0, c1;
-              load8_unaligned(region, off + 5 + 8 * i, c0, c1);
-              decode_word<FMT>(c0, lo, hi, words);
-              decode_word<FMT>(c1, lo, hi, words + 8);
-            } else {
-              uint32_t c0, c1;
-              load8_unaligned(region, off + 6 + 4 * i, c0, c1);
-              decode_word<FMT>(c0, lo, hi, words);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) words[j] = 0u;
-          }
-          const uint32_t ai = ring_it + sb;
-          const int as = ai % kRing;
-          ok = __all_sync(0xffffffffu, wait_bar(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status));
-          if (!ok) break;
-          tc_fence_after();
-          tmem_st16(tmem + lane_addr + kRingCol + as * (kMT * kSlotCols) + tile * kSlotCols, words);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh->full_a[as]);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->empty_raw[rs]);
-      }
-      raw_it += nblk;
-      ring_it += nsub;
-      if (!ok) break;
-
-      // epilogue
-      ok = __all_sync(0xffffffffu, wait_bar(&sh->acc_full, u_it & 1, sh, w.status));
-      if (!ok) break;
+    for (int ui = 0; ui < my_units; ++ui) {
+      const int4 un = units[blockIdx.x + ui * gridDim.x];
+      const int buf = ui & 1;
+      if (!wait_bar_warp(&sh->acc_full[buf], (ui / kAccBufs) & 1, sh, w.status)) break;
       tc_fence_after();
       const int cnt = un.w, n0 = un.z;
-      const int npad = max(16, (cnt + 15) & ~15);
-      for (int cc = grp; cc < npad / 16; cc += 4) {
+      const uint32_t acc0 = tmem + lane_addr + buf * (kMT * kNT);
+      for (int cc = 0; cc * 16 < cnt; ++cc) {
         uint32_t a0[16], a1[16];
-        tmem_ld16(tmem + lane_addr + 0 * kNT + cc * 16, a0);
-        tmem_ld16(tmem + lane_addr + 1 * kNT + cc * 16, a1);
+        tmem_ld16(acc0 + cc * 16, a0);
+        tmem_ld16(acc0 + kNT + cc * 16, a1);
         tmem_wait_ld();
         if (GATEUP) {
           const int rr = un.y * 128 + r;
           if (rr < d.I) {
             const int pos = perm_pos_k<FMT>(rr);
+            __half* hp = w.h16 + (size_t)(n0 + cc * 16) * d.I + pos;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const int n = cc * 16 + j;
-              if (n < cnt) {
+              if (cc * 16 + j < cnt) {
                 const float g = __uint_as_float(a0[j]);
                 const float uu = __uint_as_float(a1[j]);
-                const float hv = g / (1.0f + __expf(-g)) * uu;
-                w.h16[(size_t)(n0 + n) * d.I + pos] = __float2half_rn(hv);
+                hp[(size_t)j * d.I] = __float2half_rn(g / (1.0f + __expf(-g)) * uu);
               }
             }
           }
@@ -578,8 +496,112 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->acc_empty);
+      if (lane == 0) mbar_arrive(&sh->acc_empty[buf]);
     }
+  } else {
+    // ---------------------------------------- raw fetch + decoders -------
+    const int dw = warp - kDecWarp0;          // 0..15
+    const int grp = dw >> 2;                  // 0..3
+    const int tile = grp & 1, parity = grp >> 1;
+    const int q = warp & 3;                   // TMEM lane quarter
+    const int r = q * 32 + lane;              // lane = row inside the tile
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const int total_blocks = my_units * nblk;
+    bool ok = true;
+
+    // Fetch raw block c (linear over this CTA's units) of the 32 rows of
+    // this warp's (tile, quarter) into its stage; called by the warps whose
+    // parity equals c's.
+    auto fetch = [&](int c) -> bool {
+      const int s = c % kRawStages;
+      if (!wait_bar_warp(&sh->empty_raw[s], ((c / kRawStages) & 1) ^ 1, sh, w.status)) return false;
+      const int ui = c / nblk, kb = c % nblk;
+      const int4 un = units[blockIdx.x + ui * gridDim.x];
+      const uint8_t* blob = tab.p[un.x];
+      uint8_t* stage = raw_base + s * raw_stage_bytes<FMT>() + (tile * 128 + q * 32) * PITCH;
+#pragma unroll
+      for (int i = 0; i < CHUNKS; ++i) {
+        const int slot = i * 32 + lane;
+        const int row = slot / CHUNKS, ch = slot % CHUNKS;
+        int R;
+        const uint8_t* rp = tile_row<GATEUP>(d, blob, un.y, tile, q * 32 + row, gu_rowbytes, rowbytes, &R);
+        const uintptr_t b0 = reinterpret_cast<uintptr_t>(rp + (size_t)kb * BB);
+        const uintptr_t a0 = b0 & ~(uintptr_t)15;
+        const int nch = (int)(((b0 + BB + 15) & ~(uintptr_t)15) - a0) >> 4;
+        if (R < rows_total && ch < nch)
+          cp_async16(stage + row * PITCH + ch * 16, reinterpret_cast<const void*>(a0 + 16 * ch));
+      }
+      cp_async_mbar_arrive(&sh->full_raw[s]);
+      return true;
+    };
+
+    for (int c = 0; c < kRawAhead && c < total_blocks; ++c)
+      if ((c & 1) == parity && !fetch(c)) { ok = false; break; }
+
+    int pending = -1;                          // ring slot whose tcgen05.st is in flight
+    uint32_t ring_it = 0;
+    auto flush = [&]() {
+      if (pending >= 0) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->full_a[pending]);
+        pending = -1;
+      }
+    };
+
+    for (int c = 0; c < total_blocks && ok; ++c) {
+      const int cn = c + kRawAhead;
+      if (cn < total_blocks && (cn & 1) == parity && !fetch(cn)) { ok = false; break; }
+      const int ui = c / nblk, kb = c % nblk;
+      const int4 un = units[blockIdx.x + ui * gridDim.x];
+      const uint8_t* blob = tab.p[un.x];
+      int R;
+      const uint8_t* rowg = tile_row<GATEUP>(d, blob, un.y, tile, r, gu_rowbytes, rowbytes, &R);
+      const bool valid = R < rows_total;
+      flush();
+      const int rs = c % kRawStages;
+      if (!wait_bar_warp(&sh->full_raw[rs], (c / kRawStages) & 1, sh, w.status)) { ok = false; break; }
+      const uint8_t* region = raw_base + rs * raw_stage_bytes<FMT>() + (tile * 128 + r) * PITCH;
+      const int off = (int)(reinterpret_cast<uintptr_t>(rowg + (size_t)kb * BB) & 15);
+      uint32_t h0, h1;
+      load8_unaligned(region, off, h0, h1);
+      const float dd = half_bits_to_float(h0 & 0xffffu);
+      const uint32_t S = (h0 >> 16) | ((h1 & 0xffu) << 16);
+      const uint32_t flags = (h1 >> 8) & 0xffu;
+      for (int i = parity; i < 8; i += 2) {
+        const int sb = kb * 8 + i;
+        if (sb >= nsub) break;
+        uint32_t words[16];
+        if (valid) {
+          uint32_t lo, hi;
+          make_lut<FMT>(dd, S, flags, i, lo, hi);
+          uint32_t c0, c1;
+          if constexpr (FMT == RL_FMT_Q2) {
+            load8_unaligned(region, off + 5 + 8 * i, c0, c1);
+            decode_word<FMT>(c0, lo, hi, words);
+            decode_word<FMT>(c1, lo, hi, words + 8);
+          } else {
+            load8_unaligned(region, off + 6 + 4 * i, c0, c1);
+            decode_word<FMT>(c0, lo, hi, words);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) words[j] = 0u;
+        }
+        flush();
+        const uint32_t ai = ring_it + sb;
+        const int as = ai % kRing;
+        if (!wait_bar_warp(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st16(tmem + lane_addr + kRingCol + as * (kMT * kSlotCols) + tile * kSlotCols, words);
+        pending = as;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->empty_raw[rs]);
+      if (kb == nblk - 1) ring_it += nsub;
+    }
+    flush();
   }
 
   tc_fence_before();

@@ -134,7 +134,8 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
   mark(0, s);
   rl::route_kernel<FMT><<<d.W, 1024, 0, s>>>(logits, static_cast<const uint16_t*>(x), d, w);
   mark(1, s);
-  rl::group_kernel<<<1, 1024, 0, s>>>(d, w, 1);
+  rl::count_scan_kernel<<<1, 1024, 0, s>>>(d, w, 1);
+  rl::scatter_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w);
   mark(2, s);
   if (g_gemm == 1) {
     rl::gateup_simt_kernel<FMT><<<d.max_units_gu, 256, 0, s>>>(d, w, tab);
@@ -255,7 +256,8 @@ int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx,
   w.pair_pos = pair_pos;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   rl::route_kernel<RL_FMT_Q2><<<d.W, 1024, 0, s>>>(router_logits, nullptr, d, w);
-  rl::group_kernel<<<1, 1024, 0, s>>>(d, w, 0);
+  rl::count_scan_kernel<<<1, 1024, 0, s>>>(d, w, 0);
+  rl::scatter_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return RL_OK;
@@ -308,7 +310,7 @@ const char* rl_moe_profile_stage_name(int i) {
   return (i >= 0 && i < kStages) ? kStageNames[i] : "";
 }
 
-int rl_moe_launches_per_call(void) { return kStages; }
+int rl_moe_launches_per_call(void) { return kStages + 1; }
 
 int rl_moe_debug_set_gemm(int which) {
   if (which != 0 && which != 1) return fail(RL_ERR_INVALID_ARG, "gemm %d", which);

@@ -149,22 +149,31 @@ __device__ __forceinline__ int block_excl_scan(int v, int* swarp, int* total) {
   return base + x - v;
 }
 
-// One CTA of 1024 threads: per-expert counts from the bitmap, offsets by an
-// exclusive scan, the stable scatter (ascending token inside an expert; a
-// token picks an expert at most once), and the work lists of the two
-// decode-GEMM stages.  Deterministic: no result depends on atomics order.
-__global__ void __launch_bounds__(1024) group_kernel(Dims d, Work w, int make_units) {
+// Counts, offsets and work lists: one CTA of 1024 threads.
+//  - counts[e] = popcount of bitmap row e; every thread takes a strided slice
+//    of the flattened [E][W] bitmap (many loads in flight) and adds into
+//    shared memory (integer adds: the result does not depend on their order);
+//  - offsets = exclusive scan of the counts;
+//  - work units of the two decode-GEMM stages, expert by expert.
+__global__ void __launch_bounds__(1024) count_scan_kernel(Dims d, Work w, int make_units) {
   __shared__ int scount[kMaxE];
-  __shared__ int soff[kMaxE + 1];
   __shared__ int swarp[32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  for (int e = warp; e < d.E; e += 32) {
-    int c = 0;
-    for (int q = lane; q < d.W; q += 32) c += __popc(w.bitmap[(size_t)e * d.W + q]);
+  for (int e = threadIdx.x; e < d.E; e += blockDim.x) scount[e] = 0;
+  __syncthreads();
+  const int nwords = d.E * d.W;
+  constexpr int U = 8;
+  for (int base = threadIdx.x; base < nwords; base += U * blockDim.x) {
+    unsigned m[U];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-    if (lane == 0) scount[e] = c;
+    for (int i = 0; i < U; ++i) {
+      const int q = base + i * blockDim.x;
+      m[i] = q < nwords ? __ldg(w.bitmap + q) : 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < U; ++i) {
+      const int q = base + i * blockDim.x;
+      if (m[i]) atomicAdd(&scount[q / d.W], __popc(m[i]));
+    }
   }
   __syncthreads();
 
@@ -172,71 +181,70 @@ __global__ void __launch_bounds__(1024) group_kernel(Dims d, Work w, int make_un
   const int c = e < d.E ? scount[e] : 0;
   int total = 0;
   const int off = block_excl_scan(c, swarp, &total);
-  if (e < d.E) {
-    soff[e] = off;
-    w.offsets[e] = off;
-  }
+  if (e < d.E) w.offsets[e] = off;
   if (e == 0) {
-    soff[d.E] = total;
     w.offsets[d.E] = total;
     if (total != d.P) set_status(w.status, RL_DEV_BAD_GROUPING);
   }
-
-  if (make_units) {
-    const int ch_gu = (c + d.nt_gu - 1) / d.nt_gu;
-    const int ch_dn = (c + d.nt_dn - 1) / d.nt_dn;
-    int tot_gu = 0, tot_dn = 0;
-    const int base_gu = block_excl_scan(ch_gu * d.slabs_gu, swarp, &tot_gu);
-    const int base_dn = block_excl_scan(ch_dn * d.groups_dn, swarp, &tot_dn);
-    if (e == 0) {
-      const bool over = tot_gu > d.max_units_gu || tot_dn > d.max_units_dn;
-      if (over) set_status(w.status, RL_DEV_UNIT_OVERFLOW);
-      w.counters[0] = over ? 0 : tot_gu;
-      w.counters[1] = over ? 0 : tot_dn;
+  if (!make_units) return;
+  const int ch_gu = (c + d.nt_gu - 1) / d.nt_gu;
+  const int ch_dn = (c + d.nt_dn - 1) / d.nt_dn;
+  int tot_gu = 0, tot_dn = 0;
+  const int base_gu = block_excl_scan(ch_gu * d.slabs_gu, swarp, &tot_gu);
+  const int base_dn = block_excl_scan(ch_dn * d.groups_dn, swarp, &tot_dn);
+  const bool over = tot_gu > d.max_units_gu || tot_dn > d.max_units_dn;
+  if (e == 0) {
+    if (over) set_status(w.status, RL_DEV_UNIT_OVERFLOW);
+    w.counters[0] = over ? 0 : tot_gu;
+    w.counters[1] = over ? 0 : tot_dn;
+  }
+  if (e < d.E && !over) {
+    int q = base_gu;
+    for (int ch = 0; ch < ch_gu; ++ch) {
+      const int n0 = off + ch * d.nt_gu;
+      const int n = min(d.nt_gu, c - ch * d.nt_gu);
+      for (int s = 0; s < d.slabs_gu; ++s) w.units_gu[q++] = make_int4(e, s, n0, n);
     }
-    if (e < d.E && tot_gu <= d.max_units_gu && tot_dn <= d.max_units_dn) {
-      int q = base_gu;
-      for (int ch = 0; ch < ch_gu; ++ch) {
-        const int n0 = off + ch * d.nt_gu;
-        const int n = min(d.nt_gu, c - ch * d.nt_gu);
-        for (int s = 0; s < d.slabs_gu; ++s) w.units_gu[q++] = make_int4(e, s, n0, n);
-      }
-      q = base_dn;
-      for (int ch = 0; ch < ch_dn; ++ch) {
-        const int n0 = off + ch * d.nt_dn;
-        const int n = min(d.nt_dn, c - ch * d.nt_dn);
-        for (int s = 0; s < d.groups_dn; ++s) w.units_dn[q++] = make_int4(e, s, n0, n);
-      }
+    q = base_dn;
+    for (int ch = 0; ch < ch_dn; ++ch) {
+      const int n0 = off + ch * d.nt_dn;
+      const int n = min(d.nt_dn, c - ch * d.nt_dn);
+      for (int s = 0; s < d.groups_dn; ++s) w.units_dn[q++] = make_int4(e, s, n0, n);
     }
   }
-  __syncthreads();
+}
 
-  // Scatter: warp per expert; lanes take consecutive bitmap words.
-  for (int ex = warp; ex < d.E; ex += 32) {
-    int running = soff[ex];
-    for (int q0 = 0; q0 < d.W; q0 += 32) {
-      const int q = q0 + lane;
-      unsigned m = q < d.W ? w.bitmap[(size_t)ex * d.W + q] : 0u;
-      const int cnt = __popc(m);
-      int incl = cnt;
+// Stable scatter: one warp per expert, lanes over consecutive bitmap words;
+// pair_list[offsets[e] + r] = t*k + j for the r-th token t (ascending) that
+// chose e, and pair_pos is its inverse.  A token picks an expert at most
+// once, so ascending token is ascending pair id.
+__global__ void __launch_bounds__(256) scatter_kernel(Dims d, Work w) {
+  const int ex = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (ex >= d.E) return;
+  int running = __ldg(w.offsets + ex);
+  for (int q0 = 0; q0 < d.W; q0 += 32) {
+    const int q = q0 + lane;
+    unsigned m = q < d.W ? __ldg(w.bitmap + (size_t)ex * d.W + q) : 0u;
+    const int cnt = __popc(m);
+    int incl = cnt;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int pos = running + incl - cnt;
-      while (m) {
-        const int b = __ffs(m) - 1;
-        m &= m - 1;
-        const int t = 32 * q + b;
-        const int j = w.jslot[(size_t)ex * d.T + t];
-        const int pid = t * d.k + j;
-        w.pair_list[pos] = pid;
-        w.pair_pos[pid] = pos;
-        ++pos;
-      }
-      running += __shfl_sync(0xffffffffu, incl, 31);
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
+    int pos = running + incl - cnt;
+    while (m) {
+      const int b = __ffs(m) - 1;
+      m &= m - 1;
+      const int t = 32 * q + b;
+      const int j = w.jslot[(size_t)ex * d.T + t];
+      const int pid = t * d.k + j;
+      w.pair_list[pos] = pid;
+      w.pair_pos[pid] = pos;
+      ++pos;
+    }
+    running += __shfl_sync(0xffffffffu, incl, 31);
   }
 }
 
