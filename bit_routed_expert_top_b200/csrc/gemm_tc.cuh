@@ -149,20 +149,28 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// D[tmem] (+)= A[tmem] * B[smem], fp16 x fp16 -> fp32, cta_group::1.
+// D[tmem] (+)= A[tmem] * B[smem], fp16 x fp16 -> fp32, cta_group::1.  Called
+// by a whole converged warp with warp-uniform operands; one elected lane
+// issues (operands then live in uniform registers: issuing from a divergent
+// single lane measured ~2x slower per instruction).
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Arrive on bar when every MMA issued so far by this warp has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_addr(bar))
-               : "memory");
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_addr(bar))
+      : "memory");
 }
 
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B fp16
@@ -348,52 +356,50 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
 
   if (warp == 0) {
     // ------------------------------------------------------------ MMA ---
-    if (lane == 0) {
-      uint32_t ring_it = 0, b_it = 0;
-      bool ok = true;
-      for (int ui = 0; ui < my_units && ok; ++ui) {
-        const int4 un = units[blockIdx.x + ui * gridDim.x];
-        const int npad = max(16, (un.w + 15) & ~15);
-        const uint32_t idesc = idesc_f16(128, npad);
-        const int buf = ui & 1;
-        if (ui >= kAccBufs) ok = wait_bar(&sh->acc_empty[buf], ((ui / kAccBufs) - 1) & 1, sh, w.status);
-        tc_fence_after();
-        const uint32_t acc0 = tmem + buf * (kMT * kNT);
-        for (int sb = 0; sb < nsub && ok; ++sb) {
-          const uint32_t bi = b_it + sb / (kBK / kSubVals);
-          const int bs = bi % kBStages;
-          if (sb % (kBK / kSubVals) == 0) {
-            ok = wait_bar(&sh->full_b[bs], (bi / kBStages) & 1, sh, w.status);
-            if (!ok) break;
-          }
-          const uint32_t ai = ring_it + sb;
-          const int as = ai % kRing;
-          ok = wait_bar(&sh->full_a[as], (ai / kRing) & 1, sh, w.status);
+    // The whole warp runs this loop in lockstep; one elected lane issues.
+    uint32_t ring_it = 0, b_it = 0;
+    bool ok = true;
+    for (int ui = 0; ui < my_units && ok; ++ui) {
+      const int4 un = units[blockIdx.x + ui * gridDim.x];
+      const int npad = max(16, (un.w + 15) & ~15);
+      const uint32_t idesc = idesc_f16(128, npad);
+      const int buf = ui & 1;
+      if (ui >= kAccBufs) ok = wait_bar_warp(&sh->acc_empty[buf], ((ui / kAccBufs) - 1) & 1, sh, w.status);
+      tc_fence_after();
+      const uint32_t acc0 = tmem + buf * (kMT * kNT);
+      for (int sb = 0; sb < nsub && ok; ++sb) {
+        const uint32_t bi = b_it + sb / (kBK / kSubVals);
+        const int bs = bi % kBStages;
+        if (sb % (kBK / kSubVals) == 0) {
+          ok = wait_bar_warp(&sh->full_b[bs], (bi / kBStages) & 1, sh, w.status);
           if (!ok) break;
-          tc_fence_after();
-          const uint32_t bstage = smem_addr(b_base + bs * kBStageBytes);
-          const int kin = (sb % (kBK / kSubVals)) * kSubVals;   // K offset inside the B stage
-#pragma unroll
-          for (int t = 0; t < kMT; ++t) {
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              const uint32_t a_tm = tmem + kRingCol + as * (kMT * kSlotCols) + t * kSlotCols + kk * 8;
-              const uint64_t bd = sdesc_noswizzle(bstage + ((kin + kk * 16) / 8) * kBLbo, kBLbo, 128);
-              mma_ts(acc0 + t * kNT, a_tm, bd, idesc, (sb | kk) != 0);
-            }
-          }
-          mma_commit(&sh->empty_a[as]);
-          if (sb % (kBK / kSubVals) == (kBK / kSubVals) - 1 || sb == nsub - 1) mma_commit(&sh->empty_b[bs]);
         }
-        if (ok) mma_commit(&sh->acc_full[buf]);
-        ring_it += nsub;
-        b_it += nbchunk;
+        const uint32_t ai = ring_it + sb;
+        const int as = ai % kRing;
+        ok = wait_bar_warp(&sh->full_a[as], (ai / kRing) & 1, sh, w.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t bstage = smem_addr(b_base + bs * kBStageBytes);
+        const int kin = (sb % (kBK / kSubVals)) * kSubVals;   // K offset inside the B stage
+#pragma unroll
+        for (int t = 0; t < kMT; ++t) {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint32_t a_tm = tmem + kRingCol + as * (kMT * kSlotCols) + t * kSlotCols + kk * 8;
+            const uint64_t bd = sdesc_noswizzle(bstage + ((kin + kk * 16) / 8) * kBLbo, kBLbo, 128);
+            mma_ts(acc0 + t * kNT, a_tm, bd, idesc, (sb | kk) != 0);
+          }
+        }
+        mma_commit(&sh->empty_a[as]);
+        if (sb % (kBK / kSubVals) == (kBK / kSubVals) - 1 || sb == nsub - 1) mma_commit(&sh->empty_b[bs]);
       }
-      // drain: every MMA issued by this thread has completed before teardown
-      mma_commit(&sh->drain);
-      wait_bar(&sh->drain, 0, sh, w.status);
+      if (ok) mma_commit(&sh->acc_full[buf]);
+      ring_it += nsub;
+      b_it += nbchunk;
     }
-    __syncwarp();
+    // drain: every MMA issued by this warp has completed before teardown
+    mma_commit(&sh->drain);
+    wait_bar_warp(&sh->drain, 0, sh, w.status);
   } else if (warp == 1) {
     // ------------------------------------------- B operand gather --------
     uint32_t b_it = 0;
