@@ -47,9 +47,10 @@ constexpr int kNtDn = kNT;       // down unit size in pairs
 constexpr int kMtDn = 2;         // 128-row slabs per down unit
 constexpr int kMT = 2;           // M tiles per unit (gate+up, or two down slabs)
 constexpr int kAccBufs = 2;      // accumulator buffers (epilogue overlap)
-constexpr int kRing = 8;         // A sub-block stages in TMEM
+constexpr int kStepVals = 64;    // K values per decode step (two sub-blocks)
+constexpr int kRing = 4;         // A step stages in TMEM
 constexpr int kRingCol = kAccBufs * kMT * kNT;  // first ring column (256)
-constexpr int kSlotCols = 16;                   // 32 fp16 of K per lane
+constexpr int kSlotCols = 32;                   // 64 fp16 of K per lane
 constexpr int kRawStages = 4;
 constexpr int kRawAhead = 2;                    // raw blocks fetched ahead
 constexpr int kBStages = 4;
@@ -63,6 +64,7 @@ constexpr int kWarps = 22;
 constexpr int kThreads = kWarps * 32;
 constexpr long long kWaitCycles = 4000000000LL; // ~2 s at 2 GHz
 static_assert(kRingCol + kRing * kMT * kSlotCols <= 512, "TMEM columns");
+static_assert(kMT == 2, "the MMA issue below is written for two M tiles");
 
 template <int FMT> struct Raw;
 // row region: the 16-byte chunks that hold one block (<= 69+15 / 38+15 bytes),
@@ -134,6 +136,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+      "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -276,6 +289,26 @@ __device__ __forceinline__ void load8_unaligned(const uint8_t* region, int o, ui
   w1 = __funnelshift_r(x1, x2, s);
 }
 
+// 16 bytes starting at byte offset o of a shared-memory row region.
+__device__ __forceinline__ void load16_unaligned(const uint8_t* region, int o, uint32_t (&wv)[4]) {
+  const int u = o & ~7;
+  const uint2 a = *reinterpret_cast<const uint2*>(region + u);
+  const uint2 b = *reinterpret_cast<const uint2*>(region + u + 8);
+  const uint2 c = *reinterpret_cast<const uint2*>(region + u + 16);
+  const int sh = o & 7;
+  const bool hi4 = sh >= 4;
+  const uint32_t x0 = hi4 ? a.y : a.x;
+  const uint32_t x1 = hi4 ? b.x : a.y;
+  const uint32_t x2 = hi4 ? b.y : b.x;
+  const uint32_t x3 = hi4 ? c.x : b.y;
+  const uint32_t x4 = hi4 ? c.y : c.x;
+  const uint32_t s = (uint32_t)(sh & 3) * 8u;
+  wv[0] = __funnelshift_r(x0, x1, s);
+  wv[1] = __funnelshift_r(x1, x2, s);
+  wv[2] = __funnelshift_r(x2, x3, s);
+  wv[3] = __funnelshift_r(x3, x4, s);
+}
+
 // Rows of a unit.  GATEUP: unit {expert, slab, n0, cnt}: tile 0 = gate rows
 // 128*slab + r, tile 1 = up rows 128*slab + r, K = H.  DOWN: unit
 // {expert, group, n0, cnt}: tile t = down rows 128*(2*group+t) + r, K = I.
@@ -307,14 +340,20 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
   constexpr int BB = Fmt<FMT>::kBytes;
   constexpr int PITCH = Raw<FMT>::kPitch;
   constexpr int CHUNKS = Raw<FMT>::kChunks;
-  const int n_units = w.counters[GATEUP ? 0 : 1];
+  // the unit count is read from memory: broadcast it from lane 0 so that
+  // every loop bound derived from it is provably warp-uniform
+  const int n_units = __shfl_sync(0xffffffffu, w.counters[GATEUP ? 0 : 1], 0);
   if ((int)blockIdx.x >= n_units) return;
   const int4* units = GATEUP ? w.units_gu : w.units_dn;
   const int my_units = (n_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // warp index via a lane-0 shuffle: provably warp-uniform, so the MMA
+  // warp's loop counters and operands stay in uniform registers
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
+  const int lane = threadIdx.x & 31;
   const int K = GATEUP ? d.H : d.I;
   const int nsub = K / kSubVals;
+  const int nstep = (nsub + 1) / 2;
   const int nblk = GATEUP ? d.nbH : d.nbI;
   const int nbchunk = (K + kBK - 1) / kBK;
   const size_t rowbytes = (size_t)nblk * BB;
@@ -352,49 +391,56 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = sh->tmem_base;
+  const uint32_t tmem = __shfl_sync(0xffffffffu, sh->tmem_base, 0);
 
   if (warp == 0) {
     // ------------------------------------------------------------ MMA ---
     // The whole warp runs this loop in lockstep; one elected lane issues.
     uint32_t ring_it = 0, b_it = 0;
     bool ok = true;
+    const uint64_t bdesc0 = sdesc_noswizzle(smem_addr(b_base), kBLbo, 128);
     for (int ui = 0; ui < my_units && ok; ++ui) {
-      const int4 un = units[blockIdx.x + ui * gridDim.x];
-      const int npad = max(16, (un.w + 15) & ~15);
+      const int cnt = __shfl_sync(0xffffffffu, units[blockIdx.x + ui * gridDim.x].w, 0);
+      const int npad = max(16, (cnt + 15) & ~15);
       const uint32_t idesc = idesc_f16(128, npad);
       const int buf = ui & 1;
       if (ui >= kAccBufs) ok = wait_bar_warp(&sh->acc_empty[buf], ((ui / kAccBufs) - 1) & 1, sh, w.status);
       tc_fence_after();
       const uint32_t acc0 = tmem + buf * (kMT * kNT);
-      for (int sb = 0; sb < nsub && ok; ++sb) {
-        const uint32_t bi = b_it + sb / (kBK / kSubVals);
+      for (int st = 0; st < nstep && ok; ++st) {
+        constexpr int kStepsPerB = kBK / kStepVals;
+        const uint32_t bi = b_it + st / kStepsPerB;
         const int bs = bi % kBStages;
-        if (sb % (kBK / kSubVals) == 0) {
+        if (st % kStepsPerB == 0) {
           ok = wait_bar_warp(&sh->full_b[bs], (bi / kBStages) & 1, sh, w.status);
           if (!ok) break;
         }
-        const uint32_t ai = ring_it + sb;
+        const uint32_t ai = ring_it + st;
         const int as = ai % kRing;
         ok = wait_bar_warp(&sh->full_a[as], (ai / kRing) & 1, sh, w.status);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t bstage = smem_addr(b_base + bs * kBStageBytes);
-        const int kin = (sb % (kBK / kSubVals)) * kSubVals;   // K offset inside the B stage
-#pragma unroll
-        for (int t = 0; t < kMT; ++t) {
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const uint32_t a_tm = tmem + kRingCol + as * (kMT * kSlotCols) + t * kSlotCols + kk * 8;
-            const uint64_t bd = sdesc_noswizzle(bstage + ((kin + kk * 16) / 8) * kBLbo, kBLbo, 128);
-            mma_ts(acc0 + t * kNT, a_tm, bd, idesc, (sb | kk) != 0);
-          }
+        // B descriptor = stage base + K offset (both in 16-byte units of the address field)
+        const int kin = (st % kStepsPerB) * kStepVals;
+        const uint64_t bd = bdesc0 + (uint64_t)((bs * kBStageBytes + (kin / 8) * kBLbo) >> 4);
+        const uint32_t a_tm = tmem + kRingCol + as * (kMT * kSlotCols);
+        constexpr uint64_t kK16 = (uint64_t)(2 * kBLbo) >> 4;   // +16 K values in B
+        const uint32_t first = st == 0 ? 0u : 1u;
+        mma_ts(acc0, a_tm, bd, idesc, first);
+        mma_ts(acc0 + kNT, a_tm + kSlotCols, bd, idesc, first);
+        mma_ts(acc0, a_tm + 8, bd + kK16, idesc, 1u);
+        mma_ts(acc0 + kNT, a_tm + kSlotCols + 8, bd + kK16, idesc, 1u);
+        if (2 * st + 1 < nsub) {
+          mma_ts(acc0, a_tm + 16, bd + 2 * kK16, idesc, 1u);
+          mma_ts(acc0 + kNT, a_tm + kSlotCols + 16, bd + 2 * kK16, idesc, 1u);
+          mma_ts(acc0, a_tm + 24, bd + 3 * kK16, idesc, 1u);
+          mma_ts(acc0 + kNT, a_tm + kSlotCols + 24, bd + 3 * kK16, idesc, 1u);
         }
         mma_commit(&sh->empty_a[as]);
-        if (sb % (kBK / kSubVals) == (kBK / kSubVals) - 1 || sb == nsub - 1) mma_commit(&sh->empty_b[bs]);
+        if (st % kStepsPerB == kStepsPerB - 1 || st == nstep - 1) mma_commit(&sh->empty_b[bs]);
       }
       if (ok) mma_commit(&sh->acc_full[buf]);
-      ring_it += nsub;
+      ring_it += nstep;
       b_it += nbchunk;
     }
     // drain: every MMA issued by this warp has completed before teardown
@@ -575,37 +621,44 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
       const float dd = half_bits_to_float(h0 & 0xffffu);
       const uint32_t S = (h0 >> 16) | ((h1 & 0xffu) << 16);
       const uint32_t flags = (h1 >> 8) & 0xffu;
-      for (int i = parity; i < 8; i += 2) {
-        const int sb = kb * 8 + i;
-        if (sb >= nsub) break;
-        uint32_t words[16];
+      // steps 4*kb .. 4*kb+3 of this block; this warp takes those of its parity
+      for (int j = parity; j < 4; j += 2) {
+        const int st = kb * 4 + j;
+        if (2 * st >= nsub) break;
+        const int i = 2 * j;                   // first sub-block of the step inside the block
+        uint32_t words[32];
         if (valid) {
-          uint32_t lo, hi;
-          make_lut<FMT>(dd, S, flags, i, lo, hi);
-          uint32_t c0, c1;
+          uint32_t lo0, hi0, lo1, hi1;
+          make_lut<FMT>(dd, S, flags, i, lo0, hi0);
+          make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
           if constexpr (FMT == RL_FMT_Q2) {
-            load8_unaligned(region, off + 5 + 8 * i, c0, c1);
-            decode_word<FMT>(c0, lo, hi, words);
-            decode_word<FMT>(c1, lo, hi, words + 8);
+            uint32_t cw[4];
+            load16_unaligned(region, off + 5 + 8 * i, cw);
+            decode_word<FMT>(cw[0], lo0, hi0, words);
+            decode_word<FMT>(cw[1], lo0, hi0, words + 8);
+            decode_word<FMT>(cw[2], lo1, hi1, words + 16);
+            decode_word<FMT>(cw[3], lo1, hi1, words + 24);
           } else {
+            uint32_t c0, c1;
             load8_unaligned(region, off + 6 + 4 * i, c0, c1);
-            decode_word<FMT>(c0, lo, hi, words);
+            decode_word<FMT>(c0, lo0, hi0, words);
+            decode_word<FMT>(c1, lo1, hi1, words + 16);
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) words[j] = 0u;
+          for (int q2 = 0; q2 < 32; ++q2) words[q2] = 0u;
         }
         flush();
-        const uint32_t ai = ring_it + sb;
+        const uint32_t ai = ring_it + st;
         const int as = ai % kRing;
         if (!wait_bar_warp(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status)) { ok = false; break; }
         tc_fence_after();
-        tmem_st16(tmem + lane_addr + kRingCol + as * (kMT * kSlotCols) + tile * kSlotCols, words);
+        tmem_st32(tmem + lane_addr + kRingCol + as * (kMT * kSlotCols) + tile * kSlotCols, words);
         pending = as;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->empty_raw[rs]);
-      if (kb == nblk - 1) ring_it += nsub;
+      if (kb == nblk - 1) ring_it += nstep;
     }
     flush();
   }
