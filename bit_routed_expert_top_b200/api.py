@@ -27,6 +27,7 @@ SIGNATURES = {
     "rl_moe_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "rl_moe_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp]),
     "rl_moe_prefill_ws": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "rl_moe_prefill_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp]),
     "rl_moe_route": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "rl_moe_check_status": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_uint)]),
     "rl_moe_profile_enable": (_i, [_i]),
@@ -143,6 +144,15 @@ def rl_moe_prefill_ws(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, wor
     _check(load().rl_moe_prefill_ws(_ptr(x), _ptr(router_logits), ctypes.cast(table, ctypes.c_void_p),
                                     fmt, T, H, I, E, k, _ptr(y), _ptr(workspace), nbytes,
                                     _stream(stream)))
+
+
+def rl_moe_prefill_noalloc(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, stream=None):
+    """The layer with the library's fixed device scratch instead of a workspace
+    (no allocation on any call; see include/rl_moe.h for its limits)."""
+    _need_cuda(x, router_logits, y)
+    table = expert_blobs if isinstance(expert_blobs, ctypes.Array) else expert_table(expert_blobs, E)
+    _check(load().rl_moe_prefill_noalloc(_ptr(x), _ptr(router_logits), ctypes.cast(table, ctypes.c_void_p),
+                                         fmt, T, H, I, E, k, _ptr(y), _stream(stream)))
 
 
 def rl_moe_route(router_logits, T, E, k, topk_idx, topk_w, offsets, pair_list, pair_pos,

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "common.cuh"
@@ -170,6 +171,17 @@ int fill_table(const void* const* blobs, int E, rl::ExpertTable* tab) {
   return RL_OK;
 }
 
+// ---- fixed scratch for rl_moe_prefill_noalloc ------------------------------
+// A file-scope device array, so that the entry point below never allocates.
+// Every GPU that loads this library holds it (RL_NOALLOC_SCRATCH_BYTES) until
+// the process exits.  In host code the array's name is only a host-side
+// handle: its device address is looked up with cudaGetSymbolAddress, once per
+// device, with that device current.
+__device__ __align__(256) unsigned char g_noalloc_scratch[RL_NOALLOC_SCRATCH_BYTES];
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
 }  // namespace
 
 extern "C" {
@@ -232,6 +244,39 @@ int rl_moe_prefill(const void* x, const float* router_logits, const void* const*
   if (rc != RL_OK) return rc;
   if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
   return RL_OK;
+}
+
+int rl_moe_prefill_noalloc(const void* x, const float* router_logits,
+                           const void* const* expert_blobs, int fmt, int T, int H, int I, int E,
+                           int k, float* y, void* stream) {
+  rl::Dims d;
+  Layout L;
+  int rc = plan(fmt, T, H, I, E, k, &d, &L);
+  if (rc != RL_OK) return rc;
+  if (T == 0) return RL_OK;
+  if (L.total > RL_NOALLOC_SCRATCH_BYTES)
+    return fail(RL_ERR_UNSUPPORTED,
+                "these sizes need %zu bytes of scratch, more than the fixed %zu bytes of "
+                "rl_moe_prefill_noalloc; use rl_moe_prefill_ws with a caller workspace",
+                L.total, (size_t)RL_NOALLOC_SCRATCH_BYTES);
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(RL_ERR_UNSUPPORTED, "device %d >= %d", dev, kMaxDevices);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+      e = cudaGetSymbolAddress(&g_noalloc_addr[dev], g_noalloc_scratch);
+      if (e != cudaSuccess) {
+        g_noalloc_addr[dev] = nullptr;
+        return cuda_fail(e, "cudaGetSymbolAddress(fixed scratch)");
+      }
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  return rl_moe_prefill_ws(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, scratch,
+                           RL_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx, float* topk_w,

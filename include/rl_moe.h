@@ -115,6 +115,37 @@ int rl_moe_prefill_ws(const void* x, const float* router_logits,
                       int I, int E, int k, float* y, void* workspace,
                       size_t ws_bytes, void* stream);
 
+/* Fixed size of the scratch array used by rl_moe_prefill_noalloc (16 MiB). */
+#define RL_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * rl_moe_prefill without any device allocation (the Red Lite pages have no
+ * counterpart of this entry point).  For callers that cannot call cudaMalloc
+ * or cudaMallocAsync: code that runs while a CUDA graph is being captured in a
+ * mode that forbids allocation, engines that have handed all device memory to
+ * their own pool, and decode / verify loops that cannot afford an allocation
+ * (which may synchronize the device) on every step.
+ *
+ * Same arguments and result as rl_moe_prefill.  Instead of a workspace it
+ * uses one fixed array of RL_NOALLOC_SCRATCH_BYTES in device memory that the
+ * library defines; every GPU that loads the library holds it until the
+ * process exits.  Sizes whose workspace (rl_moe_workspace_bytes) exceeds that
+ * return RL_ERR_UNSUPPORTED with a message; this covers small chunks such as
+ * the 2-token verify step, not a 2,048-token prefill.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, and it keeps the last call's
+ *     contents: calls that overlap on the GPU (other streams, other threads)
+ *     race and corrupt each other's results.  Order them on one stream.
+ *   - The device status word lives in the shared array and cannot be read
+ *     through this entry point; use rl_moe_prefill_ws when it is needed.
+ * The function calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+int rl_moe_prefill_noalloc(const void* x, const float* router_logits,
+                           const void* const* expert_blobs, int fmt, int T, int H, int I,
+                           int E, int k, float* y, void* stream);
+
 /*
  * Steps 1-2 alone (parity/debug export).  Outputs, all device memory:
  *   topk_idx int32 [T, k], topk_w fp32 [T, k]  (selection order)
