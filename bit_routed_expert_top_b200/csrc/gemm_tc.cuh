@@ -41,19 +41,33 @@
 namespace rl {
 namespace tc {
 
-constexpr int kNT = 64;          // max pairs per unit = accumulator columns per tile
+// Tuning knobs (compile-time; the defaults are the measured best).
+#ifndef RL_TC_NT
+#define RL_TC_NT 64
+#endif
+#ifndef RL_TC_RAW_STAGES
+#define RL_TC_RAW_STAGES 4
+#endif
+#ifndef RL_TC_RAW_AHEAD
+#define RL_TC_RAW_AHEAD 2
+#endif
+#ifndef RL_TC_B_STAGES
+#define RL_TC_B_STAGES 4
+#endif
+constexpr int kNT = RL_TC_NT;    // max pairs per unit = accumulator columns per tile
 constexpr int kNtGu = kNT;       // gate/up unit size in pairs
 constexpr int kNtDn = kNT;       // down unit size in pairs
 constexpr int kMtDn = 2;         // 128-row slabs per down unit
 constexpr int kMT = 2;           // M tiles per unit (gate+up, or two down slabs)
 constexpr int kAccBufs = 2;      // accumulator buffers (epilogue overlap)
 constexpr int kStepVals = 64;    // K values per decode step (two sub-blocks)
-constexpr int kRing = 4;         // A step stages in TMEM
-constexpr int kRingCol = kAccBufs * kMT * kNT;  // first ring column (256)
+constexpr int kRingSlotCols = 2 * 32;                                   // both tiles, 64 K values
+constexpr int kRingCol = kAccBufs * kMT * kNT;  // first ring column
+constexpr int kRing = (512 - kRingCol) / kRingSlotCols;                 // A step stages in TMEM
 constexpr int kSlotCols = 32;                   // 64 fp16 of K per lane
-constexpr int kRawStages = 4;
-constexpr int kRawAhead = 2;                    // raw blocks fetched ahead
-constexpr int kBStages = 4;
+constexpr int kRawStages = RL_TC_RAW_STAGES;
+constexpr int kRawAhead = RL_TC_RAW_AHEAD;      // raw blocks fetched ahead
+constexpr int kBStages = RL_TC_B_STAGES;
 constexpr int kBK = 128;                        // K values per B stage
 constexpr int kBLbo = (kNT / 8) * 128;          // bytes between K core matrices (1024)
 constexpr int kBStageBytes = (kBK / 8) * kBLbo; // 16 KB
@@ -63,6 +77,8 @@ constexpr int kDecWarp0 = 6;
 constexpr int kWarps = 22;
 constexpr int kThreads = kWarps * 32;
 constexpr long long kWaitCycles = 4000000000LL; // ~2 s at 2 GHz
+constexpr int kUnitCache = 64;                  // this CTA's first work units, cached in shared memory
+constexpr int kSharedBytes = 4096;              // barriers, work-unit cache, pair tokens
 static_assert(kRingCol + kRing * kMT * kSlotCols <= 512, "TMEM columns");
 static_assert(kMT == 2, "the MMA issue below is written for two M tiles");
 
@@ -77,7 +93,7 @@ __host__ __device__ constexpr int raw_stage_bytes() { return kRows * Raw<FMT>::k
 
 template <int FMT>
 __host__ __device__ constexpr int smem_bytes() {
-  return kRawStages * raw_stage_bytes<FMT>() + kBStages * kBStageBytes + 1024;
+  return kRawStages * raw_stage_bytes<FMT>() + kBStages * kBStageBytes + kSharedBytes;
 }
 
 // ------------------------------------------------------------------ PTX ---
@@ -90,10 +106,30 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
+// arrive only where pred is true, without a branch
+__device__ __forceinline__ void mbar_arrive_if(uint64_t* bar, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+      "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_addr(bar)),
+      "r"((uint32_t)pred)
+      : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
                "r"(bytes)
                : "memory");
+}
+// Non-blocking test of a phase (issued ahead of the work it guards).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   uint32_t ok;
@@ -136,6 +172,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -200,6 +242,7 @@ __device__ __forceinline__ uint64_t sdesc_noswizzle(uint32_t saddr, uint32_t lbo
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
+
 struct Shared {
   uint64_t full_raw[kRawStages], empty_raw[kRawStages];
   uint64_t full_b[kBStages], empty_b[kBStages];
@@ -208,14 +251,22 @@ struct Shared {
   uint32_t tmem_base;
   int abort_flag;
   int toks[kNT];
+  int4 unit[kUnitCache];                 // units blockIdx.x + i*gridDim.x
+  const uint8_t* blob[kUnitCache];       // their expert blobs
 };
+static_assert(sizeof(Shared) + 16 <= kSharedBytes, "shared-memory control block");
 
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared* sh, unsigned* status) {
+// Bounded wait.  Roles whose waits are long (epilogue, B gather) pass
+// sleepy=true and back off with nanosleep, leaving issue slots to the
+// decoder warps on the same scheduler; the MMA and decoder warps spin.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared* sh, unsigned* status,
+                                         bool sleepy = false) {
   const uint32_t addr = smem_addr(bar);
   long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(addr, parity)) return true;
-    if ((it & 31u) == 31u) {
+    if (sleepy) __nanosleep(256);
+    if (sleepy || (it & 15u) == 15u) {
       if (*(volatile int*)&sh->abort_flag) return false;
       const long long now = clock64();
       if (t0 == 0) {
@@ -229,8 +280,10 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared*
   }
 }
 // Warp-uniform variant: every lane waits, the result is agreed with a vote.
-__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, Shared* sh, unsigned* status) {
-  return __all_sync(0xffffffffu, wait_bar(bar, parity, sh, status));
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, Shared* sh, unsigned* status,
+                                              bool sleepy = false) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(smem_addr(bar), parity))) return true;
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, sh, status, sleepy));
 }
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
@@ -260,16 +313,34 @@ __device__ __forceinline__ void make_lut(float dd, uint32_t S, uint32_t flags, i
 // One 32-bit code word -> fp16x2 words out[0 .. G/2).  Word 2k+h holds the
 // values (k + 2h*P, k + (2h+1)*P) of the group, P = codes per byte, i.e.
 // position i holds value (i >> 2) + P*(i & 3).
+//
+// Per four codes: one LOP3 (mask) and two PRMT on the integer ALU pipe, and
+// the shifts and selector arithmetic as multiplies on the FMA pipe
+// (x >> n = mulhi(x, 2^(32-n)); the selector of bytes 2-3 is a mad.hi), so
+// the two pipes share the work.
+__device__ __forceinline__ uint32_t mulhi_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t madhi_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
 template <int FMT>
 __device__ __forceinline__ void decode_word(uint32_t c, uint32_t lo, uint32_t hi, uint32_t* out) {
   constexpr int P = Fmt<FMT>::kPerByte;
+  constexpr int B = Fmt<FMT>::kBits;
   constexpr uint32_t mask = FMT == RL_FMT_Q2 ? 0x03030303u : 0x01010101u;
 #pragma unroll
   for (int k = 0; k < P; ++k) {
-    const uint32_t v = (c >> (Fmt<FMT>::kBits * k)) & mask;
-    const uint32_t sel = v * 0x22u + 0x10101010u;
-    out[2 * k] = __byte_perm(lo, hi, sel);
-    out[2 * k + 1] = __byte_perm(lo, hi, sel >> 16);
+    const uint32_t shifted = k == 0 ? c : mulhi_u32(c, 1u << (32 - B * k));
+    const uint32_t v = shifted & mask;
+    const uint32_t sel_lo = v * 0x22u + 0x10101010u;          // selectors of bytes 0-1
+    const uint32_t sel_hi = madhi_u32(v, 0x00220000u, 0x1010u); // selectors of bytes 2-3
+    out[2 * k] = __byte_perm(lo, hi, sel_lo);
+    out[2 * k + 1] = __byte_perm(lo, hi, sel_hi);
   }
 }
 
@@ -360,6 +431,11 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
   const size_t gu_rowbytes = (size_t)d.nbH * BB;
   const int rows_total = GATEUP ? d.I : d.H;
 
+  for (int i = threadIdx.x; i < my_units && i < kUnitCache; i += blockDim.x) {
+    const int4 un = units[blockIdx.x + i * gridDim.x];
+    sh->unit[i] = un;
+    sh->blob[i] = tab.p[un.x];
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRawStages; ++s) {
       mbar_init(&sh->full_raw[s], 8 * 32);   // 8 fetching warps x 32 lanes (cp.async arrivals)
@@ -392,6 +468,13 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = __shfl_sync(0xffffffffu, sh->tmem_base, 0);
+  // work unit ui of this CTA and its expert blob (shared-memory cache first)
+  auto unit_at = [&](int ui) -> int4 {
+    return ui < kUnitCache ? sh->unit[ui] : units[blockIdx.x + ui * gridDim.x];
+  };
+  auto blob_at = [&](int ui, int e) -> const uint8_t* {
+    return ui < kUnitCache ? sh->blob[ui] : tab.p[e];
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ MMA ---
@@ -400,7 +483,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
     bool ok = true;
     const uint64_t bdesc0 = sdesc_noswizzle(smem_addr(b_base), kBLbo, 128);
     for (int ui = 0; ui < my_units && ok; ++ui) {
-      const int cnt = __shfl_sync(0xffffffffu, units[blockIdx.x + ui * gridDim.x].w, 0);
+      const int cnt = __shfl_sync(0xffffffffu, unit_at(ui).w, 0);
       const int npad = max(16, (cnt + 15) & ~15);
       const uint32_t idesc = idesc_f16(128, npad);
       const int buf = ui & 1;
@@ -452,7 +535,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
     bool ok = true;
     int pending = -1;                      // stage whose copies are in flight
     for (int ui = 0; ui < my_units && ok; ++ui) {
-      const int4 un = units[blockIdx.x + ui * gridDim.x];
+      const int4 un = unit_at(ui);
       const int cnt = un.w, n0 = un.z;
       const int npad = max(16, (cnt + 15) & ~15);
       // the previous unit's last stage must land before toks is rewritten
@@ -469,7 +552,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
       const __half* src_base = GATEUP ? w.x16 : w.h16;
       for (int kc = 0; kc < nbchunk && ok; ++kc, ++b_it) {
         const int s = b_it % kBStages;
-        ok = wait_bar_warp(&sh->empty_b[s], ((b_it / kBStages) & 1) ^ 1, sh, w.status);
+        ok = wait_bar_warp(&sh->empty_b[s], ((b_it / kBStages) & 1) ^ 1, sh, w.status, true);
         if (!ok) break;
         uint8_t* stage = b_base + s * kBStageBytes;
         const int kbase = kc * kBK;
@@ -507,9 +590,9 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
     const int r = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     for (int ui = 0; ui < my_units; ++ui) {
-      const int4 un = units[blockIdx.x + ui * gridDim.x];
+      const int4 un = unit_at(ui);
       const int buf = ui & 1;
-      if (!wait_bar_warp(&sh->acc_full[buf], (ui / kAccBufs) & 1, sh, w.status)) break;
+      if (!wait_bar_warp(&sh->acc_full[buf], (ui / kAccBufs) & 1, sh, w.status, true)) break;
       tc_fence_after();
       const int cnt = un.w, n0 = un.z;
       const uint32_t acc0 = tmem + lane_addr + buf * (kMT * kNT);
@@ -528,7 +611,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
               if (cc * 16 + j < cnt) {
                 const float g = __uint_as_float(a0[j]);
                 const float uu = __uint_as_float(a1[j]);
-                hp[(size_t)j * d.I] = __float2half_rn(g / (1.0f + __expf(-g)) * uu);
+                hp[(size_t)j * d.I] = __float2half_rn(__fdividef(g * uu, 1.0f + __expf(-g)));
               }
             }
           }
@@ -557,31 +640,41 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
     const int tile = grp & 1, parity = grp >> 1;
     const int q = warp & 3;                   // TMEM lane quarter
     const int r = q * 32 + lane;              // lane = row inside the tile
-    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const uint32_t a_col = tmem + ((uint32_t)(q * 32) << 16) + kRingCol + tile * kSlotCols;
+    uint8_t* const my_region0 = raw_base + (tile * 128 + r) * PITCH;
     const int total_blocks = my_units * nblk;
     bool ok = true;
 
-    // Fetch raw block c (linear over this CTA's units) of the 32 rows of
-    // this warp's (tile, quarter) into its stage; called by the warps whose
-    // parity equals c's.
+    // Per-unit address of this thread's row (block 0).  The fetching lane
+    // of a row is the row's own thread (lane = row).
+    int cur_ui = -1;
+    const uint8_t* rowg = nullptr;
+    auto row_of_unit = [&](int ui) {
+      if (ui == cur_ui) return;
+      cur_ui = ui;
+      const int4 un = unit_at(ui);
+      int R;
+      rowg = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, r, gu_rowbytes, rowbytes, &R);
+    };
+
+    // Fetch raw block c (linear over this CTA's units) of this warp's 32
+    // rows: every lane copies the 16-byte chunks that hold its own row's block.
+    // Called by the warps whose parity equals c's.
     auto fetch = [&](int c) -> bool {
       const int s = c % kRawStages;
       if (!wait_bar_warp(&sh->empty_raw[s], ((c / kRawStages) & 1) ^ 1, sh, w.status)) return false;
       const int ui = c / nblk, kb = c % nblk;
-      const int4 un = units[blockIdx.x + ui * gridDim.x];
-      const uint8_t* blob = tab.p[un.x];
-      uint8_t* stage = raw_base + s * raw_stage_bytes<FMT>() + (tile * 128 + q * 32) * PITCH;
-#pragma unroll
-      for (int i = 0; i < CHUNKS; ++i) {
-        const int slot = i * 32 + lane;
-        const int row = slot / CHUNKS, ch = slot % CHUNKS;
-        int R;
-        const uint8_t* rp = tile_row<GATEUP>(d, blob, un.y, tile, q * 32 + row, gu_rowbytes, rowbytes, &R);
-        const uintptr_t b0 = reinterpret_cast<uintptr_t>(rp + (size_t)kb * BB);
+      const int4 un = unit_at(ui);
+      int R;
+      const uint8_t* rp = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, r, gu_rowbytes, rowbytes, &R);
+      if (R < rows_total) {
+        const uintptr_t b0 = reinterpret_cast<uintptr_t>(rp) + (uintptr_t)kb * BB;
         const uintptr_t a0 = b0 & ~(uintptr_t)15;
-        const int nch = (int)(((b0 + BB + 15) & ~(uintptr_t)15) - a0) >> 4;
-        if (R < rows_total && ch < nch)
-          cp_async16(stage + row * PITCH + ch * 16, reinterpret_cast<const void*>(a0 + 16 * ch));
+        const int nch = (int)((((b0 + BB + 15) & ~(uintptr_t)15) - a0) >> 4);
+        uint8_t* dst = my_region0 + s * raw_stage_bytes<FMT>();
+#pragma unroll
+        for (int ch = 0; ch < CHUNKS; ++ch)
+          if (ch < nch) cp_async16(dst + ch * 16, reinterpret_cast<const void*>(a0 + 16 * ch));
       }
       cp_async_mbar_arrive(&sh->full_raw[s]);
       return true;
@@ -597,7 +690,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->full_a[pending]);
+        mbar_arrive_if(&sh->full_a[pending], lane == 0);
         pending = -1;
       }
     };
@@ -605,17 +698,13 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
     for (int c = 0; c < total_blocks && ok; ++c) {
       const int cn = c + kRawAhead;
       if (cn < total_blocks && (cn & 1) == parity && !fetch(cn)) { ok = false; break; }
-      const int ui = c / nblk, kb = c % nblk;
-      const int4 un = units[blockIdx.x + ui * gridDim.x];
-      const uint8_t* blob = tab.p[un.x];
-      int R;
-      const uint8_t* rowg = tile_row<GATEUP>(d, blob, un.y, tile, r, gu_rowbytes, rowbytes, &R);
-      const bool valid = R < rows_total;
+      const int ui = c / nblk, kb = c - ui * nblk;
+      row_of_unit(ui);
       flush();
       const int rs = c % kRawStages;
       if (!wait_bar_warp(&sh->full_raw[rs], (c / kRawStages) & 1, sh, w.status)) { ok = false; break; }
-      const uint8_t* region = raw_base + rs * raw_stage_bytes<FMT>() + (tile * 128 + r) * PITCH;
-      const int off = (int)(reinterpret_cast<uintptr_t>(rowg + (size_t)kb * BB) & 15);
+      const uint8_t* region = my_region0 + rs * raw_stage_bytes<FMT>();
+      const int off = (int)((reinterpret_cast<uintptr_t>(rowg) + (uintptr_t)kb * BB) & 15);
       uint32_t h0, h1;
       load8_unaligned(region, off, h0, h1);
       const float dd = half_bits_to_float(h0 & 0xffffu);
@@ -626,38 +715,42 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
         const int st = kb * 4 + j;
         if (2 * st >= nsub) break;
         const int i = 2 * j;                   // first sub-block of the step inside the block
-        uint32_t words[32];
-        if (valid) {
-          uint32_t lo0, hi0, lo1, hi1;
-          make_lut<FMT>(dd, S, flags, i, lo0, hi0);
-          make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
-          if constexpr (FMT == RL_FMT_Q2) {
-            uint32_t cw[4];
-            load16_unaligned(region, off + 5 + 8 * i, cw);
-            decode_word<FMT>(cw[0], lo0, hi0, words);
-            decode_word<FMT>(cw[1], lo0, hi0, words + 8);
-            decode_word<FMT>(cw[2], lo1, hi1, words + 16);
-            decode_word<FMT>(cw[3], lo1, hi1, words + 24);
-          } else {
-            uint32_t c0, c1;
-            load8_unaligned(region, off + 6 + 4 * i, c0, c1);
-            decode_word<FMT>(c0, lo0, hi0, words);
-            decode_word<FMT>(c1, lo1, hi1, words + 16);
-          }
-        } else {
-#pragma unroll
-          for (int q2 = 0; q2 < 32; ++q2) words[q2] = 0u;
-        }
-        flush();
         const uint32_t ai = ring_it + st;
         const int as = ai % kRing;
-        if (!wait_bar_warp(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status)) { ok = false; break; }
+        // test the ring slot now; the answer is needed only after the decode
+        const bool slot_free = mbar_test_wait(smem_addr(&sh->empty_a[as]), ((ai / kRing) & 1) ^ 1);
+        // rows past the matrix decode stale stage bytes: their accumulator
+        // rows (TMEM lanes) are never read by the epilogue
+        uint32_t words[32];
+        uint32_t lo0, hi0, lo1, hi1;
+        make_lut<FMT>(dd, S, flags, i, lo0, hi0);
+        make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
+        if constexpr (FMT == RL_FMT_Q2) {
+          uint32_t cw[4];
+          load16_unaligned(region, off + 5 + 8 * i, cw);
+          decode_word<FMT>(cw[0], lo0, hi0, words);
+          decode_word<FMT>(cw[1], lo0, hi0, words + 8);
+          decode_word<FMT>(cw[2], lo1, hi1, words + 16);
+          decode_word<FMT>(cw[3], lo1, hi1, words + 24);
+        } else {
+          uint32_t c0, c1;
+          load8_unaligned(region, off + 6 + 4 * i, c0, c1);
+          decode_word<FMT>(c0, lo0, hi0, words);
+          decode_word<FMT>(c1, lo1, hi1, words + 16);
+        }
+        flush();
+        if (!__all_sync(0xffffffffu, slot_free) &&
+            !wait_bar_warp(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status)) { ok = false; break; }
         tc_fence_after();
-        tmem_st32(tmem + lane_addr + kRingCol + as * (kMT * kSlotCols) + tile * kSlotCols, words);
+        const uint32_t dst = a_col + as * (kMT * kSlotCols);
+        tmem_st8(dst, words);
+        tmem_st8(dst + 8, words + 8);
+        tmem_st8(dst + 16, words + 16);
+        tmem_st8(dst + 24, words + 24);
         pending = as;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->empty_raw[rs]);
+      mbar_arrive_if(&sh->empty_raw[rs], lane == 0);
       if (kb == nblk - 1) ring_it += nstep;
     }
     flush();

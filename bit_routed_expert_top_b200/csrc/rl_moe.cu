@@ -129,11 +129,26 @@ inline void mark(int i, cudaStream_t s) {
 // Which decode-GEMM implementation runs (0: tensor cores, 1: CUDA cores).
 int g_gemm = 0;
 
+// Route: one CTA per 8 tokens over every byte column of the token bitmap;
+// values per lane = smallest power of two >= E/32.
+template <int FMT>
+void launch_route(const float* logits, const uint16_t* x, const rl::Dims& d, const rl::Work& w,
+                  cudaStream_t s) {
+  const int grid = d.W * 4;
+  const int per = (d.E + 31) / 32;
+  if (per <= 1) rl::route_kernel<FMT, 1><<<grid, 256, 0, s>>>(logits, x, d, w);
+  else if (per <= 2) rl::route_kernel<FMT, 2><<<grid, 256, 0, s>>>(logits, x, d, w);
+  else if (per <= 4) rl::route_kernel<FMT, 4><<<grid, 256, 0, s>>>(logits, x, d, w);
+  else if (per <= 8) rl::route_kernel<FMT, 8><<<grid, 256, 0, s>>>(logits, x, d, w);
+  else if (per <= 16) rl::route_kernel<FMT, 16><<<grid, 256, 0, s>>>(logits, x, d, w);
+  else rl::route_kernel<FMT, 32><<<grid, 256, 0, s>>>(logits, x, d, w);
+}
+
 template <int FMT>
 int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
                const rl::Work& w, float* y, cudaStream_t s) {
   mark(0, s);
-  rl::route_kernel<FMT><<<d.W, 1024, 0, s>>>(logits, static_cast<const uint16_t*>(x), d, w);
+  launch_route<FMT>(logits, static_cast<const uint16_t*>(x), d, w, s);
   mark(1, s);
   rl::count_scan_kernel<<<1, 1024, 0, s>>>(d, w, 1);
   rl::scatter_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w);
@@ -150,7 +165,7 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
     if (rc2 != RL_OK) return rc2;
   }
   mark(4, s);
-  rl::combine_kernel<<<dim3(d.T, (d.H + 1023) / 1024), 256, 0, s>>>(d, w.pw, w.o16, y);
+  rl::combine_kernel<<<dim3(d.T, (d.H + 1023) / 1024), 128, 0, s>>>(d, w.pw, w.o16, y);
   mark(5, s);
   if (g_prof) g_ev_recorded = true;
   const cudaError_t e = cudaGetLastError();
@@ -300,7 +315,7 @@ int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx,
   w.pair_list = pair_list;
   w.pair_pos = pair_pos;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  rl::route_kernel<RL_FMT_Q2><<<d.W, 1024, 0, s>>>(router_logits, nullptr, d, w);
+  launch_route<RL_FMT_Q2>(router_logits, nullptr, d, w, s);
   rl::count_scan_kernel<<<1, 1024, 0, s>>>(d, w, 0);
   rl::scatter_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w);
   const cudaError_t e = cudaGetLastError();

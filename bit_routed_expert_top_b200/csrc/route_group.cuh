@@ -22,55 +22,66 @@ __device__ __forceinline__ bool route_better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-// One CTA of 1024 threads handles 32 consecutive tokens (one bitmap word
-// column); warp w handles token 32*blockIdx.x + w.
-//  - top-k by k rounds of a warp-wide arg-max over the not-yet-taken experts;
-//  - z_j = expf(l_j - l_0) summed in j order, p_j = z_j / sum;
-//  - the CTA's 32-bit token mask of every expert is built in shared memory
-//    and written to bitmap[e][blockIdx.x] in full (no zeroing pass needed);
-//  - with x != nullptr, the warp also writes its token's x row as fp16 in the
-//    K-permuted order of format FMT (one conversion per token, reused by all
-//    of its k experts).
-template <int FMT>
-__global__ void __launch_bounds__(1024)
-route_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ x,
-             Dims d, Work w) {
+// One CTA of 8 warps handles 8 consecutive tokens (one byte column of the
+// token bitmap); warp w handles token 8*blockIdx.x + w.  The grid covers
+// every byte column of the bitmap (4 per 32-bit word), so CTAs past T write
+// zero bytes and no zeroing pass is needed.
+//  - Lane l holds the logits of experts l, l+32, ... (PER per lane, PER a
+//    power of two >= E/32) and its best not-yet-taken one.  Each of the k
+//    rounds takes the warp-wide best of the lanes' bests (larger value, or
+//    equal value and lower expert index; -0.0 equals +0.0); only the winning
+//    lane rescans its own values.
+//  - z_j = expf(l_j - l_0) summed in j order, p_j = z_j / sum.
+//  - With x != nullptr the warp also writes its token's x row as fp16 in the
+//    K-permuted order of format FMT.
+template <int FMT, int PER>
+__global__ void __launch_bounds__(256)
+route_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ x, Dims d, Work w) {
   __shared__ unsigned smask[kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 32 + warp;
+  const int t = blockIdx.x * 8 + warp;
   if (blockIdx.x == 0 && threadIdx.x == 0) w.status[0] = 0u;
   for (int e = threadIdx.x; e < d.E; e += blockDim.x) smask[e] = 0u;
   __syncthreads();
 
   if (t < d.T) {
     const float* row = logits + (size_t)t * d.E;
-    const int per = (d.E + 31) >> 5;
-    float v[kMaxE / 32];
+    float v[PER];
     unsigned taken = 0u;
 #pragma unroll
-    for (int m = 0; m < kMaxE / 32; ++m) {
+    for (int m = 0; m < PER; ++m) {
       const int e = lane + 32 * m;
-      if (m < per && e < d.E) v[m] = __ldg(row + e);
+      if (e < d.E) v[m] = __ldg(row + e);
       else { v[m] = 0.f; taken |= 1u << m; }
     }
+    // this lane's best untaken entry
+    auto rescan = [&](float& bv, int& bi) {
+      bv = 0.f;
+      bi = -1;
+#pragma unroll
+      for (int m = 0; m < PER; ++m) {
+        const bool free_m = !((taken >> m) & 1u);
+        // strict '>' keeps the lower index on equal values (m ascending)
+        if (free_m && (bi < 0 || v[m] > bv)) { bv = v[m]; bi = lane + 32 * m; }
+      }
+    };
+    float mv;
+    int mi;
+    rescan(mv, mi);
     float l0 = 0.f, sum = 0.f;
     for (int j = 0; j < d.k; ++j) {
-      float bv = 0.f;
-      int bi = -1;
-#pragma unroll
-      for (int m = 0; m < kMaxE / 32; ++m) {
-        if (!((taken >> m) & 1u) && route_better(v[m], lane + 32 * m, bv, bi)) {
-          bv = v[m];
-          bi = lane + 32 * m;
-        }
-      }
+      float bv = mv;
+      int bi = mi;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
         const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
         if (route_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
       }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if ((bi & 31) == lane) {
+        taken |= 1u << (bi >> 5);
+        rescan(mv, mi);
+      }
       if (j == 0) l0 = bv;
       const float z = expf(bv - l0);
       sum += z;                                   // same value in every lane
@@ -118,8 +129,10 @@ route_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ x,
     }
   }
   __syncthreads();
+  uint8_t* bm8 = reinterpret_cast<uint8_t*>(w.bitmap);
+  const size_t row_bytes = (size_t)d.W * 4;
   for (int e = threadIdx.x; e < d.E; e += blockDim.x)
-    w.bitmap[(size_t)e * d.W + blockIdx.x] = smask[e];
+    bm8[(size_t)e * row_bytes + blockIdx.x] = (uint8_t)smask[e];
 }
 
 // Exclusive scan of one int per thread over a 1024-thread block.
@@ -249,24 +262,44 @@ __global__ void __launch_bounds__(256) scatter_kernel(Dims d, Work w) {
 }
 
 // Step 5: y[t, c] = sum_j p_{t,j} o_{t*k+j}[c], added in selection order j.
+// 8 columns per thread (16-byte loads), slots loaded four at a time ahead of
+// their fp32 fused multiply-adds, which run in j order.
 __global__ void __launch_bounds__(256)
 combine_kernel(Dims d, const float* __restrict__ pw, const __half* __restrict__ o16,
                float* __restrict__ y) {
   const int t = blockIdx.x;
-  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
   if (c >= d.H) return;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  for (int j = 0; j < d.k; ++j) {
-    const float p = __ldg(pw + (size_t)t * d.k + j);
-    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(o16 + ((size_t)t * d.k + j) * d.H + c));
-    const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-    const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-    a0 = fmaf(p, lo.x, a0);
-    a1 = fmaf(p, lo.y, a1);
-    a2 = fmaf(p, hi.x, a2);
-    a3 = fmaf(p, hi.y, a3);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  const size_t base = (size_t)t * d.k;
+  for (int j0 = 0; j0 < d.k; j0 += 4) {
+    uint4 raw[4];
+    float p[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      if (j0 + jj < d.k) {
+        raw[jj] = __ldg(reinterpret_cast<const uint4*>(o16 + (base + j0 + jj) * d.H + c));
+        p[jj] = __ldg(pw + base + j0 + jj);
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      if (j0 + jj < d.k) {
+        const uint32_t wv[4] = {raw[jj].x, raw[jj].y, raw[jj].z, raw[jj].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[q]));
+          acc[2 * q] = fmaf(p[jj], f.x, acc[2 * q]);
+          acc[2 * q + 1] = fmaf(p[jj], f.y, acc[2 * q + 1]);
+        }
+      }
+    }
   }
-  *reinterpret_cast<float4*>(y + (size_t)t * d.H + c) = make_float4(a0, a1, a2, a3);
+  float4* yo = reinterpret_cast<float4*>(y + (size_t)t * d.H + c);
+  yo[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  yo[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
 }  // namespace rl
