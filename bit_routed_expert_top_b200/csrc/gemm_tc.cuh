@@ -17,15 +17,17 @@
 //   * M = 128 weight rows, N = the unit's pairs rounded up to 16 (the pages'
 //     32-pair tiles lost because the partial tile wasted matrix work, dev72
 //     section 4; here the waste is at most 15 columns), K = 16 per MMA;
-//   * B = the unit's activation rows (x for gate/up, h for down) gathered
-//     into shared memory in the canonical no-swizzle K-major layout;
+//   * B = the unit's activation rows (x for gate/up, h for down) brought into
+//     shared memory by TMA in the 128-byte-swizzled K-major layout;
 //   * gate and up are two M tiles of one unit sharing B, so both run in one
 //     pass (two passes over the pairs lost on the pages, dev76 section 3),
 //     and the SwiGLU runs in the epilogue on the two TMEM accumulators.
 //
 // Warp roles (22 warps, one CTA per SM, persistent over the unit list):
 //   warp 0       TMEM allocation and the single MMA-issuing thread
-//   warp 1       B operand gather (16-byte cp.async into the K-major layout)
+//   warp 1       B operand by TMA, one elected thread: tile::gather4 of the
+//                pairs' x rows (gate/up) or a 2D tile of h rows (down), into
+//                the 128-byte-swizzled K-major layout
 //   warps 2..5   epilogue (one per TMEM lane quarter), double-buffered
 //                accumulators so it overlaps the next unit's MMAs
 //   warps 6..21  16 decoders: 4 groups = 2 M tiles x 2 sub-block parities,
@@ -35,6 +37,8 @@
 // Every wait is bounded: on timeout the CTA raises RL_DEV_WAIT_TIMEOUT in
 // the status word and all roles leave their loops.
 #pragma once
+
+#include <cuda.h>
 
 #include "common.cuh"
 
@@ -69,8 +73,9 @@ constexpr int kRawStages = RL_TC_RAW_STAGES;
 constexpr int kRawAhead = RL_TC_RAW_AHEAD;      // raw blocks fetched ahead
 constexpr int kBStages = RL_TC_B_STAGES;
 constexpr int kBK = 128;                        // K values per B stage
-constexpr int kBLbo = (kNT / 8) * 128;          // bytes between K core matrices (1024)
-constexpr int kBStageBytes = (kBK / 8) * kBLbo; // 16 KB
+constexpr int kBKBlock = 64;                    // K values per 128-byte swizzled row
+constexpr int kBBlockBytes = kNT * 128;         // one K block: kNT rows x 128 bytes
+constexpr int kBStageBytes = (kBK / kBKBlock) * kBBlockBytes;
 constexpr int kRows = kMT * 128;                // weight rows per unit
 constexpr int kEpiWarp0 = 2;
 constexpr int kDecWarp0 = 6;
@@ -87,6 +92,8 @@ template <int FMT> struct Raw;
 // pitch an odd number of 16-byte chunks
 template <> struct Raw<RL_FMT_Q2> { static constexpr int kPitch = 112; static constexpr int kChunks = 6; };
 template <> struct Raw<RL_FMT_Q1> { static constexpr int kPitch = 80; static constexpr int kChunks = 4; };
+static_assert((kRawStages * kRows * 112) % 1024 == 0 && (kRawStages * kRows * 80) % 1024 == 0,
+              "B stages must start 1024-byte aligned (128-byte swizzle)");
 
 template <int FMT>
 __host__ __device__ constexpr int raw_stage_bytes() { return kRows * Raw<FMT>::kPitch; }
@@ -147,6 +154,23 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+// TMA: 2D tile load and 4-row gather load into shared memory, completion
+// counted in bytes on an mbarrier (no multicast).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int y0, int y1, int y2,
+                                            int y3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5, %6}], [%7];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_addr(bar))
       : "memory");
 }
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -234,14 +258,15 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 __device__ __forceinline__ uint32_t idesc_f16(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-// Shared-memory matrix descriptor, no swizzle, K-major: start address,
-// leading byte offset (next 8-value core matrix along K), stride byte offset
-// (next group of 8 rows along N), all >> 4; version 1 in bits 46-47.
-__device__ __forceinline__ uint64_t sdesc_noswizzle(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
-}
 
+
+// Shared-memory matrix descriptor, 128-byte swizzle, K-major: rows of 128
+// bytes (64 fp16 of K), 8-row atoms 1024 bytes apart (stride byte offset);
+// the leading byte offset is unused in this mode (set to 16 bytes).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
 
 struct Shared {
   uint64_t full_raw[kRawStages], empty_raw[kRawStages];
@@ -402,7 +427,7 @@ __device__ __forceinline__ const uint8_t* tile_row(const Dims& d, const uint8_t*
 
 template <int FMT, bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
+decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUtensorMap bmap) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* raw_base = smem_raw;
   uint8_t* b_base = raw_base + kRawStages * raw_stage_bytes<FMT>();
@@ -481,7 +506,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
     // The whole warp runs this loop in lockstep; one elected lane issues.
     uint32_t ring_it = 0, b_it = 0;
     bool ok = true;
-    const uint64_t bdesc0 = sdesc_noswizzle(smem_addr(b_base), kBLbo, 128);
+    const uint64_t bdesc0 = sdesc_sw128(smem_addr(b_base));
     for (int ui = 0; ui < my_units && ok; ++ui) {
       const int cnt = __shfl_sync(0xffffffffu, unit_at(ui).w, 0);
       const int npad = max(16, (cnt + 15) & ~15);
@@ -503,11 +528,11 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
         ok = wait_bar_warp(&sh->full_a[as], (ai / kRing) & 1, sh, w.status);
         if (!ok) break;
         tc_fence_after();
-        // B descriptor = stage base + K offset (both in 16-byte units of the address field)
-        const int kin = (st % kStepsPerB) * kStepVals;
-        const uint64_t bd = bdesc0 + (uint64_t)((bs * kBStageBytes + (kin / 8) * kBLbo) >> 4);
+        // B descriptor = stage base + K block of this step; +32 bytes per 16 K
+        // values inside the swizzled 128-byte rows (address field in 16 B units)
+        const uint64_t bd = bdesc0 + (uint64_t)((bs * kBStageBytes + (st % kStepsPerB) * kBBlockBytes) >> 4);
         const uint32_t a_tm = tmem + kRingCol + as * (kMT * kSlotCols);
-        constexpr uint64_t kK16 = (uint64_t)(2 * kBLbo) >> 4;   // +16 K values in B
+        constexpr uint64_t kK16 = 32 >> 4;
         const uint32_t first = st == 0 ? 0u : 1u;
         mma_ts(acc0, a_tm, bd, idesc, first);
         mma_ts(acc0 + kNT, a_tm + kSlotCols, bd, idesc, first);
@@ -530,59 +555,46 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
     mma_commit(&sh->drain);
     wait_bar_warp(&sh->drain, 0, sh, w.status);
   } else if (warp == 1) {
-    // ------------------------------------------- B operand gather --------
+    // ------------------------------------------- B operand by TMA --------
+    // Lane 0 posts the byte count; the lanes then issue the copies in parallel
+    // (gather4: lane l takes rows 4l..4l+3); the warp stays converged.
     uint32_t b_it = 0;
     bool ok = true;
-    int pending = -1;                      // stage whose copies are in flight
     for (int ui = 0; ui < my_units && ok; ++ui) {
       const int4 un = unit_at(ui);
       const int cnt = un.w, n0 = un.z;
       const int npad = max(16, (cnt + 15) & ~15);
-      // the previous unit's last stage must land before toks is rewritten
-      if (pending >= 0) {
-        cp_async_wait<0>();
-        fence_proxy_async();
+      if (GATEUP) {
+        // token of each pair (padding rows repeat the first pair's token)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->full_b[pending]);
-        pending = -1;
+        for (int n = lane; n < npad; n += 32)
+          sh->toks[n] = w.pair_list[n0 + (n < cnt ? n : 0)] / d.k;
+        __syncwarp();
       }
-      for (int n = lane; n < cnt; n += 32)
-        sh->toks[n] = GATEUP ? w.pair_list[n0 + n] / d.k : n0 + n;
-      __syncwarp();
-      const __half* src_base = GATEUP ? w.x16 : w.h16;
       for (int kc = 0; kc < nbchunk && ok; ++kc, ++b_it) {
         const int s = b_it % kBStages;
         ok = wait_bar_warp(&sh->empty_b[s], ((b_it / kBStages) & 1) ^ 1, sh, w.status, true);
         if (!ok) break;
         uint8_t* stage = b_base + s * kBStageBytes;
-        const int kbase = kc * kBK;
-        const int kvalid = min(kBK, K - kbase);
-        for (int g8 = 0; g8 < npad / 8; ++g8) {
-          const int n = g8 * 8 + (lane & 7);
-          const int tok = n < cnt ? sh->toks[n] : 0;
-          const __half* rowp = src_base + (size_t)tok * K + kbase;
+        const int rows = GATEUP ? npad : kNT;
+        if (lane == 0)
+          mbar_arrive_expect_tx(&sh->full_b[s], (uint32_t)((kBK / kBKBlock) * rows * 128));
+        __syncwarp();
+        if (GATEUP) {
+          // lane l gathers rows 4l..4l+3 of both K blocks
+          const int n = 4 * lane;
+          if (n < npad) {
+            const int t0 = sh->toks[n], t1 = sh->toks[n + 1], t2 = sh->toks[n + 2], t3 = sh->toks[n + 3];
 #pragma unroll
-          for (int quad = 0; quad < kBK / 32; ++quad) {
-            const int c = quad * 4 + (lane >> 3);          // 8-value chunk inside the stage
-            if (n < cnt && c * 8 < kvalid)
-              cp_async16(stage + c * kBLbo + g8 * 128 + (lane & 7) * 16, rowp + c * 8);
+            for (int kb2 = 0; kb2 < kBK / kBKBlock; ++kb2)
+              tma_gather4(stage + kb2 * kBBlockBytes + n * 128, &bmap, kc * kBK + kb2 * kBKBlock, t0, t1, t2, t3,
+                          &sh->full_b[s]);
           }
+        } else if (lane < kBK / kBKBlock) {
+          tma_load_2d(stage + lane * kBBlockBytes, &bmap, kc * kBK + lane * kBKBlock, n0, &sh->full_b[s]);
         }
-        cp_async_commit();
-        if (pending >= 0) {
-          cp_async_wait<1>();
-          fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh->full_b[pending]);
-        }
-        pending = s;
+        __syncwarp();
       }
-    }
-    if (pending >= 0) {
-      cp_async_wait<0>();
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->full_b[pending]);
     }
   } else if (warp < kDecWarp0) {
     // ------------------------------------------------------ epilogue -----
@@ -667,15 +679,23 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab) {
       const int4 un = unit_at(ui);
       int R;
       const uint8_t* rp = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, r, gu_rowbytes, rowbytes, &R);
-      if (R < rows_total) {
-        const uintptr_t b0 = reinterpret_cast<uintptr_t>(rp) + (uintptr_t)kb * BB;
+      // consecutive lanes copy consecutive 16-byte chunks of one row
+      (void)rp;
+      const uint8_t* blob = blob_at(ui, un.x);
+      uint8_t* stage_w = raw_base + s * raw_stage_bytes<FMT>() + (tile * 128 + q * 32) * PITCH;
+#pragma unroll
+      for (int i2 = 0; i2 < CHUNKS; ++i2) {
+        const int slot = i2 * 32 + lane;
+        const int row = slot / CHUNKS, ch = slot - row * CHUNKS;
+        int R2;
+        const uint8_t* rp2 = tile_row<GATEUP>(d, blob, un.y, tile, q * 32 + row, gu_rowbytes, rowbytes, &R2);
+        const uintptr_t b0 = reinterpret_cast<uintptr_t>(rp2) + (uintptr_t)kb * BB;
         const uintptr_t a0 = b0 & ~(uintptr_t)15;
         const int nch = (int)((((b0 + BB + 15) & ~(uintptr_t)15) - a0) >> 4);
-        uint8_t* dst = my_region0 + s * raw_stage_bytes<FMT>();
-#pragma unroll
-        for (int ch = 0; ch < CHUNKS; ++ch)
-          if (ch < nch) cp_async16(dst + ch * 16, reinterpret_cast<const void*>(a0 + 16 * ch));
+        if (R2 < rows_total && ch < nch)
+          cp_async16(stage_w + row * PITCH + ch * 16, reinterpret_cast<const void*>(a0 + 16 * ch));
       }
+
       cp_async_mbar_arrive(&sh->full_raw[s]);
       return true;
     };
@@ -777,7 +797,7 @@ inline int num_sms() {
 }
 
 template <int FMT, bool GATEUP>
-int launch(const Dims& d, const Work& w, const ExpertTable& tab, cudaStream_t s) {
+int launch(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& bmap, cudaStream_t s) {
   static bool configured = false;
   constexpr int smem = smem_bytes<FMT>();
   if (!configured) {
@@ -788,17 +808,17 @@ int launch(const Dims& d, const Work& w, const ExpertTable& tab, cudaStream_t s)
   }
   const int maxu = GATEUP ? d.max_units_gu : d.max_units_dn;
   const int grid = maxu < num_sms() ? maxu : num_sms();
-  decode_gemm_kernel<FMT, GATEUP><<<grid, kThreads, smem, s>>>(d, w, tab);
+  decode_gemm_kernel<FMT, GATEUP><<<grid, kThreads, smem, s>>>(d, w, tab, bmap);
   return RL_OK;
 }
 
 template <int FMT>
-int launch_gateup(const Dims& d, const Work& w, const ExpertTable& tab, cudaStream_t s) {
-  return launch<FMT, true>(d, w, tab, s);
+int launch_gateup(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& xmap, cudaStream_t s) {
+  return launch<FMT, true>(d, w, tab, xmap, s);
 }
 template <int FMT>
-int launch_down(const Dims& d, const Work& w, const ExpertTable& tab, cudaStream_t s) {
-  return launch<FMT, false>(d, w, tab, s);
+int launch_down(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& hmap, cudaStream_t s) {
+  return launch<FMT, false>(d, w, tab, hmap, s);
 }
 
 }  // namespace tc

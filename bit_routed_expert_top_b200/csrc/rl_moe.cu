@@ -1,5 +1,6 @@
 // rl_moe.cu - host side of librl_moe.so: argument checks, workspace layout,
 // kernel launches and the C ABI declared in include/rl_moe.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdarg>
@@ -129,6 +130,40 @@ inline void mark(int i, cudaStream_t s) {
 // Which decode-GEMM implementation runs (0: tensor cores, 1: CUDA cores).
 int g_gemm = 0;
 
+// ---- TMA descriptors of the B operands (x16 for gate/up, h16 for down) -----
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// fp16 [rows][K] row-major, 128-byte swizzled boxes of 64 x box_rows.
+int make_act_map(CUtensorMap* map, const void* base, int K, long long rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(RL_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  const cuuint32_t es[2] = {1u, 1u};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RL_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return RL_OK;
+}
+
 // Route: one CTA per 8 tokens over every byte column of the token bitmap;
 // values per lane = smallest power of two >= E/32.
 template <int FMT>
@@ -158,11 +193,16 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
     mark(3, s);
     rl::down_simt_kernel<FMT><<<d.max_units_dn, 256, 0, s>>>(d, w, tab);
   } else {
-    const int rc = rl::tc::launch_gateup<FMT>(d, w, tab, s);
+    alignas(64) CUtensorMap xmap, hmap;
+    int rc = make_act_map(&xmap, w.x16, d.H, d.T, 1);
+    if (rc != RL_OK) return rc;
+    rc = make_act_map(&hmap, w.h16, d.I, d.P, rl::tc::kNT);
+    if (rc != RL_OK) return rc;
+    rc = rl::tc::launch_gateup<FMT>(d, w, tab, xmap, s);
     if (rc != RL_OK) return rc;
     mark(3, s);
-    const int rc2 = rl::tc::launch_down<FMT>(d, w, tab, s);
-    if (rc2 != RL_OK) return rc2;
+    rc = rl::tc::launch_down<FMT>(d, w, tab, hmap, s);
+    if (rc != RL_OK) return rc;
   }
   mark(4, s);
   rl::combine_kernel<<<dim3(d.T, (d.H + 1023) / 1024), 128, 0, s>>>(d, w.pw, w.o16, y);
