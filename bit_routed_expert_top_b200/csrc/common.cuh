@@ -19,6 +19,7 @@ constexpr int kSubVals = 32;
 constexpr int kQ2Bytes = 69;
 constexpr int kQ1Bytes = 38;
 constexpr int kMaxE = RL_MAX_EXPERTS;
+constexpr int kMaxGroupCtas = (kMaxE + 7) / 8;  // grouping CTAs: 8 experts each
 
 // Rows of one tensor-core M tile; also the row slab of a work unit.
 constexpr int kSlabRows = 128;
@@ -98,6 +99,7 @@ struct Work {
   int* pair_list;        // [P] grouped by expert, ascending token
   int* pair_pos;         // [P] inverse
   int* counters;         // [0] gate/up units, [1] down units
+  unsigned long long* look;  // [ceil(E/8)] prefix records of the grouping CTAs
   int4* units_gu;        // {expert, slab, first grouped position, pairs}
   int4* units_dn;        // {expert, slab group, first grouped position, pairs}
   __half* x16;           // [T][H] x as fp16, K-permuted per group

@@ -23,7 +23,7 @@
 //     pass (two passes over the pairs lost on the pages, dev76 section 3),
 //     and the SwiGLU runs in the epilogue on the two TMEM accumulators.
 //
-// Warp roles (22 warps, one CTA per SM, persistent over the unit list):
+// Warp roles (24 warps, one CTA per SM, persistent over the unit list):
 //   warp 0       TMEM allocation and the single MMA-issuing thread
 //   warp 1       B operand by TMA, one elected thread: tile::gather4 of the
 //                pairs' x rows (gate/up) or a 2D tile of h rows (down), into
@@ -31,9 +31,12 @@
 //   warps 2..5   epilogue (one per TMEM lane quarter), double-buffered
 //                accumulators so it overlaps the next unit's MMAs
 //   warps 6..21  16 decoders: 4 groups = 2 M tiles x 2 sub-block parities,
-//                one warp per lane quarter.  The warps of one parity also
-//                fetch the raw blocks of every other K block for their rows
-//                (16-byte cp.async, completion counted on an mbarrier).
+//                one warp per lane quarter; a step's A slot is handed to the
+//                MMA warp as soon as its TMEM stores have completed
+//   warps 22,23  raw-block fetch, one warp per M tile: 16-byte cp.async of
+//                the 128 rows' blocks (consecutive lanes copy consecutive
+//                chunks of a row), completion counted on an mbarrier, up to
+//                kRawStages K blocks ahead of the decoders
 // Every wait is bounded: on timeout the CTA raises RL_DEV_WAIT_TIMEOUT in
 // the status word and all roles leave their loops.
 #pragma once
@@ -52,9 +55,6 @@ namespace tc {
 #ifndef RL_TC_RAW_STAGES
 #define RL_TC_RAW_STAGES 4
 #endif
-#ifndef RL_TC_RAW_AHEAD
-#define RL_TC_RAW_AHEAD 2
-#endif
 #ifndef RL_TC_B_STAGES
 #define RL_TC_B_STAGES 4
 #endif
@@ -70,7 +70,6 @@ constexpr int kRingCol = kAccBufs * kMT * kNT;  // first ring column
 constexpr int kRing = (512 - kRingCol) / kRingSlotCols;                 // A step stages in TMEM
 constexpr int kSlotCols = 32;                   // 64 fp16 of K per lane
 constexpr int kRawStages = RL_TC_RAW_STAGES;
-constexpr int kRawAhead = RL_TC_RAW_AHEAD;      // raw blocks fetched ahead
 constexpr int kBStages = RL_TC_B_STAGES;
 constexpr int kBK = 128;                        // K values per B stage
 constexpr int kBKBlock = 64;                    // K values per 128-byte swizzled row
@@ -79,7 +78,8 @@ constexpr int kBStageBytes = (kBK / kBKBlock) * kBBlockBytes;
 constexpr int kRows = kMT * 128;                // weight rows per unit
 constexpr int kEpiWarp0 = 2;
 constexpr int kDecWarp0 = 6;
-constexpr int kWarps = 22;
+constexpr int kFetchWarp0 = 22;
+constexpr int kWarps = 24;
 constexpr int kThreads = kWarps * 32;
 constexpr long long kWaitCycles = 4000000000LL; // ~2 s at 2 GHz
 constexpr int kUnitCache = 64;                  // this CTA's first work units, cached in shared memory
@@ -463,7 +463,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRawStages; ++s) {
-      mbar_init(&sh->full_raw[s], 8 * 32);   // 8 fetching warps x 32 lanes (cp.async arrivals)
+      mbar_init(&sh->full_raw[s], kMT * 32); // fetch warps x 32 lanes (cp.async arrivals)
       mbar_init(&sh->empty_raw[s], 16);      // all decoder warps
     }
     for (int s = 0; s < kBStages; ++s) {
@@ -645,8 +645,8 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->acc_empty[buf]);
     }
-  } else {
-    // ---------------------------------------- raw fetch + decoders -------
+  } else if (warp < kFetchWarp0) {
+    // ------------------------------------------------------ decoders -----
     const int dw = warp - kDecWarp0;          // 0..15
     const int grp = dw >> 2;                  // 0..3
     const int tile = grp & 1, parity = grp >> 1;
@@ -657,8 +657,8 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     const int total_blocks = my_units * nblk;
     bool ok = true;
 
-    // Per-unit address of this thread's row (block 0).  The fetching lane
-    // of a row is the row's own thread (lane = row).
+    // Per-unit address of this thread's row (block 0): the offset of a block
+    // inside its 16-byte aligned copy follows from it.
     int cur_ui = -1;
     const uint8_t* rowg = nullptr;
     auto row_of_unit = [&](int ui) {
@@ -669,58 +669,10 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       rowg = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, r, gu_rowbytes, rowbytes, &R);
     };
 
-    // Fetch raw block c (linear over this CTA's units) of this warp's 32
-    // rows: every lane copies the 16-byte chunks that hold its own row's block.
-    // Called by the warps whose parity equals c's.
-    auto fetch = [&](int c) -> bool {
-      const int s = c % kRawStages;
-      if (!wait_bar_warp(&sh->empty_raw[s], ((c / kRawStages) & 1) ^ 1, sh, w.status)) return false;
-      const int ui = c / nblk, kb = c % nblk;
-      const int4 un = unit_at(ui);
-      int R;
-      const uint8_t* rp = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, r, gu_rowbytes, rowbytes, &R);
-      // consecutive lanes copy consecutive 16-byte chunks of one row
-      (void)rp;
-      const uint8_t* blob = blob_at(ui, un.x);
-      uint8_t* stage_w = raw_base + s * raw_stage_bytes<FMT>() + (tile * 128 + q * 32) * PITCH;
-#pragma unroll
-      for (int i2 = 0; i2 < CHUNKS; ++i2) {
-        const int slot = i2 * 32 + lane;
-        const int row = slot / CHUNKS, ch = slot - row * CHUNKS;
-        int R2;
-        const uint8_t* rp2 = tile_row<GATEUP>(d, blob, un.y, tile, q * 32 + row, gu_rowbytes, rowbytes, &R2);
-        const uintptr_t b0 = reinterpret_cast<uintptr_t>(rp2) + (uintptr_t)kb * BB;
-        const uintptr_t a0 = b0 & ~(uintptr_t)15;
-        const int nch = (int)((((b0 + BB + 15) & ~(uintptr_t)15) - a0) >> 4);
-        if (R2 < rows_total && ch < nch)
-          cp_async16(stage_w + row * PITCH + ch * 16, reinterpret_cast<const void*>(a0 + 16 * ch));
-      }
-
-      cp_async_mbar_arrive(&sh->full_raw[s]);
-      return true;
-    };
-
-    for (int c = 0; c < kRawAhead && c < total_blocks; ++c)
-      if ((c & 1) == parity && !fetch(c)) { ok = false; break; }
-
-    int pending = -1;                          // ring slot whose tcgen05.st is in flight
     uint32_t ring_it = 0;
-    auto flush = [&]() {
-      if (pending >= 0) {
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        mbar_arrive_if(&sh->full_a[pending], lane == 0);
-        pending = -1;
-      }
-    };
-
     for (int c = 0; c < total_blocks && ok; ++c) {
-      const int cn = c + kRawAhead;
-      if (cn < total_blocks && (cn & 1) == parity && !fetch(cn)) { ok = false; break; }
       const int ui = c / nblk, kb = c - ui * nblk;
       row_of_unit(ui);
-      flush();
       const int rs = c % kRawStages;
       if (!wait_bar_warp(&sh->full_raw[rs], (c / kRawStages) & 1, sh, w.status)) { ok = false; break; }
       const uint8_t* region = my_region0 + rs * raw_stage_bytes<FMT>();
@@ -758,7 +710,6 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
           decode_word<FMT>(c0, lo0, hi0, words);
           decode_word<FMT>(c1, lo1, hi1, words + 16);
         }
-        flush();
         if (!__all_sync(0xffffffffu, slot_free) &&
             !wait_bar_warp(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status)) { ok = false; break; }
         tc_fence_after();
@@ -767,13 +718,48 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
         tmem_st8(dst + 8, words + 8);
         tmem_st8(dst + 16, words + 16);
         tmem_st8(dst + 24, words + 24);
-        pending = as;
+        // hand the slot to the MMA warp once the stores have landed
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        mbar_arrive_if(&sh->full_a[as], lane == 0);
       }
       __syncwarp();
       mbar_arrive_if(&sh->empty_raw[rs], lane == 0);
       if (kb == nblk - 1) ring_it += nstep;
     }
-    flush();
+  } else {
+    // ----------------------------------------------------- raw fetch -----
+    // Warp kFetchWarp0 + t copies M tile t's rows.  A row's block starts at
+    // an arbitrary byte: the 16-byte chunks that hold it are copied, and the
+    // decoders find the block at the start address's offset mod 16.
+    const int tile = warp - kFetchWarp0;
+    constexpr int kCopies = 128 * CHUNKS / 32;  // cp.async per lane per block
+    bool ok = true;
+    int c = 0;
+    for (int ui = 0; ui < my_units && ok; ++ui) {
+      const int4 un = unit_at(ui);
+      int R0;
+      const uint8_t* row0 = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, 0, gu_rowbytes, rowbytes, &R0);
+      const int valid = min(128, rows_total - R0);   // rows of this tile inside the matrix
+      for (int kb = 0; kb < nblk; ++kb, ++c) {
+        const int s = c % kRawStages;
+        ok = wait_bar_warp(&sh->empty_raw[s], ((c / kRawStages) & 1) ^ 1, sh, w.status);
+        if (!ok) break;
+        uint8_t* stage = raw_base + s * raw_stage_bytes<FMT>() + tile * 128 * PITCH;
+        const uint8_t* blk0 = row0 + (size_t)kb * BB;
+#pragma unroll 6
+        for (int i2 = 0; i2 < kCopies; ++i2) {
+          const int slot = i2 * 32 + lane;
+          const int row = slot / CHUNKS, ch = slot - row * CHUNKS;
+          const uintptr_t b0 = reinterpret_cast<uintptr_t>(blk0) + (uint32_t)row * (uint32_t)rowbytes;
+          const uintptr_t a0 = (b0 & ~(uintptr_t)15) + 16 * ch;
+          if (row < valid && a0 < b0 + BB)
+            cp_async16(stage + row * PITCH + ch * 16, reinterpret_cast<const void*>(a0));
+        }
+        cp_async_mbar_arrive(&sh->full_raw[s]);
+      }
+    }
   }
 
   tc_fence_before();

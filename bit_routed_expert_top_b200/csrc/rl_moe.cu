@@ -38,9 +38,12 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 constexpr int kNtGateUp = rl::tc::kNtGu;
 constexpr int kNtDown = rl::tc::kNtDn;
 constexpr int kMtDown = rl::tc::kMtDn;
+static_assert(kNtGateUp == kNtDown, "the grouping kernel derives both unit lists from one chunk prefix");
+// route, group, gate/up, down, combine
+constexpr int kLaunchesPerCall = 5;
 
 struct Layout {
-  size_t status, idx, pw, bitmap, jslot, offsets, pair_list, pair_pos, counters,
+  size_t status, idx, pw, bitmap, jslot, offsets, pair_list, pair_pos, counters, look,
       units_gu, units_dn, x16, h16, o16, total;
 };
 
@@ -86,6 +89,7 @@ int plan(int fmt, int T, int H, int I, int E, int k, rl::Dims* d, Layout* L) {
   L->pair_list = take((size_t)d->P * 4);
   L->pair_pos = take((size_t)d->P * 4);
   L->counters = take(64);
+  L->look = take((size_t)rl::kMaxGroupCtas * 8);
   L->units_gu = take((size_t)d->max_units_gu * 16);
   L->units_dn = take((size_t)d->max_units_dn * 16);
   L->x16 = take((size_t)T * H * 2);
@@ -107,6 +111,7 @@ rl::Work carve(void* ws, const Layout& L) {
   w.pair_list = reinterpret_cast<int*>(b + L.pair_list);
   w.pair_pos = reinterpret_cast<int*>(b + L.pair_pos);
   w.counters = reinterpret_cast<int*>(b + L.counters);
+  w.look = reinterpret_cast<unsigned long long*>(b + L.look);
   w.units_gu = reinterpret_cast<int4*>(b + L.units_gu);
   w.units_dn = reinterpret_cast<int4*>(b + L.units_dn);
   w.x16 = reinterpret_cast<__half*>(b + L.x16);
@@ -185,8 +190,7 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
   mark(0, s);
   launch_route<FMT>(logits, static_cast<const uint16_t*>(x), d, w, s);
   mark(1, s);
-  rl::count_scan_kernel<<<1, 1024, 0, s>>>(d, w, 1);
-  rl::scatter_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w);
+  rl::group_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w, 1);
   mark(2, s);
   if (g_gemm == 1) {
     rl::gateup_simt_kernel<FMT><<<d.max_units_gu, 256, 0, s>>>(d, w, tab);
@@ -356,8 +360,7 @@ int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx,
   w.pair_pos = pair_pos;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   launch_route<RL_FMT_Q2>(router_logits, nullptr, d, w, s);
-  rl::count_scan_kernel<<<1, 1024, 0, s>>>(d, w, 0);
-  rl::scatter_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w);
+  rl::group_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w, 0);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return RL_OK;
@@ -410,7 +413,7 @@ const char* rl_moe_profile_stage_name(int i) {
   return (i >= 0 && i < kStages) ? kStageNames[i] : "";
 }
 
-int rl_moe_launches_per_call(void) { return kStages + 1; }
+int rl_moe_launches_per_call(void) { return kLaunchesPerCall; }
 
 int rl_moe_debug_set_gemm(int which) {
   if (which != 0 && which != 1) return fail(RL_ERR_INVALID_ARG, "gemm %d", which);

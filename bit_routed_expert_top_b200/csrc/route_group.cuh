@@ -40,7 +40,10 @@ route_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ x, D
   __shared__ unsigned smask[kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
-  if (blockIdx.x == 0 && threadIdx.x == 0) w.status[0] = 0u;
+  if (blockIdx.x == 0) {
+    if (threadIdx.x == 0) w.status[0] = 0u;
+    for (int i = threadIdx.x; i < kMaxGroupCtas; i += blockDim.x) w.look[i] = 0ull;
+  }
   for (int e = threadIdx.x; e < d.E; e += blockDim.x) smask[e] = 0u;
   __syncthreads();
 
@@ -98,33 +101,49 @@ route_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ x, D
     for (int j = lane; j < d.k; j += 32) w.pw[(size_t)t * d.k + j] *= inv;
 
     if (x != nullptr) {
+      // batches of kB groups per lane: every load of a batch is issued
+      // before the first conversion
       constexpr int G = Fmt<FMT>::kGroup;
+      constexpr int kB = 64 / G;
       const uint16_t* xr = x + (size_t)t * d.H;
       __half* xo = w.x16 + (size_t)t * d.H;
-      for (int g = lane; g < d.H / G; g += 32) {
-        uint16_t in[G];
+      const int ng = d.H / G;
+      for (int g0 = lane; g0 < ng; g0 += kB * 32) {
+        uint4 raw[kB][G / 8];
 #pragma unroll
-        for (int q = 0; q < G / 8; ++q) {
-          const uint4 v4 = __ldg(reinterpret_cast<const uint4*>(xr + g * G) + q);
-          const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+        for (int u = 0; u < kB; ++u) {
+          const int g = g0 + u * 32;
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            in[q * 8 + 2 * r] = (uint16_t)(wv[r] & 0xffffu);
-            in[q * 8 + 2 * r + 1] = (uint16_t)(wv[r] >> 16);
+          for (int q = 0; q < G / 8; ++q)
+            raw[u][q] = g < ng ? __ldg(reinterpret_cast<const uint4*>(xr + g * G) + q) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int g = g0 + u * 32;
+          if (g >= ng) break;
+          uint16_t in[G];
+#pragma unroll
+          for (int q = 0; q < G / 8; ++q) {
+            const uint32_t wv[4] = {raw[u][q].x, raw[u][q].y, raw[u][q].z, raw[u][q].w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              in[q * 8 + 2 * r] = (uint16_t)(wv[r] & 0xffffu);
+              in[q * 8 + 2 * r + 1] = (uint16_t)(wv[r] >> 16);
+            }
           }
-        }
-        uint32_t outw[G / 2];
+          uint32_t outw[G / 2];
 #pragma unroll
-        for (int c = 0; c < G / 2; ++c) {
-          const float a = __uint_as_float((uint32_t)in[perm_value<FMT>(2 * c)] << 16);
-          const float b = __uint_as_float((uint32_t)in[perm_value<FMT>(2 * c + 1)] << 16);
-          const __half2 hh = __floats2half2_rn(a, b);
-          outw[c] = *reinterpret_cast<const uint32_t*>(&hh);
-        }
+          for (int c = 0; c < G / 2; ++c) {
+            const float a = __uint_as_float((uint32_t)in[perm_value<FMT>(2 * c)] << 16);
+            const float b = __uint_as_float((uint32_t)in[perm_value<FMT>(2 * c + 1)] << 16);
+            const __half2 hh = __floats2half2_rn(a, b);
+            outw[c] = *reinterpret_cast<const uint32_t*>(&hh);
+          }
 #pragma unroll
-        for (int q = 0; q < G / 8; ++q)
-          reinterpret_cast<uint4*>(xo + g * G)[q] =
-              make_uint4(outw[4 * q], outw[4 * q + 1], outw[4 * q + 2], outw[4 * q + 3]);
+          for (int q = 0; q < G / 8; ++q)
+            reinterpret_cast<uint4*>(xo + g * G)[q] =
+                make_uint4(outw[4 * q], outw[4 * q + 1], outw[4 * q + 2], outw[4 * q + 3]);
+        }
       }
     }
   }
@@ -135,110 +154,127 @@ route_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ x, D
     bm8[(size_t)e * row_bytes + blockIdx.x] = (uint8_t)smask[e];
 }
 
-// Exclusive scan of one int per thread over a 1024-thread block.
-__device__ __forceinline__ int block_excl_scan(int v, int* swarp, int* total) {
+// Prefix record of one grouping CTA, one 64-bit word: bits 0-24 pairs,
+// bits 25-44 pair chunks (units of at most nt pairs), bits 62-63 state
+// (0 nothing yet, 1 the CTA's own sums, 2 sums including every earlier CTA).
+__device__ __forceinline__ unsigned long long look_pack(unsigned state, int pairs, int chunks) {
+  return ((unsigned long long)state << 62) | ((unsigned long long)chunks << 25) | (unsigned long long)pairs;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Step 2 in one launch of ceil(E/8) CTAs x 8 warps, warp w of CTA b owning
+// expert e = 8b + w:
+//  - count c_e = popcount of bitmap row e; chunks_e = ceil(c_e / nt);
+//  - offsets by a single-pass scan across CTAs (each CTA publishes its sums,
+//    then adds the records of the CTAs before it, walking back until one
+//    holds a full prefix; every CTA of this small grid is resident at once,
+//    and the walk is bounded);
+//  - work units of both decode-GEMM stages (nt_gu == nt_dn, so both follow
+//    from the chunk prefix);
+//  - stable scatter: pair_list[offsets[e] + r] = t*k + j for the r-th token
+//    t (ascending) that chose e, and pair_pos is its inverse.  A token picks
+//    an expert at most once, so ascending token is ascending pair id.
+// The route kernel zeroes the prefix records before this kernel runs.
+__global__ void __launch_bounds__(256) group_kernel(Dims d, Work w, int make_units) {
+  __shared__ int s_c[8], s_ch[8];
+  __shared__ int s_base_c, s_base_ch;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int x = v;
+  const int e = blockIdx.x * 8 + warp;
+  const unsigned* row = w.bitmap + (size_t)e * d.W;
+  int c = 0;
+  if (e < d.E)
+    for (int q = lane; q < d.W; q += 32) c += __popc(__ldg(row + q));
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, off);
-    if (lane >= off) x += y;
-  }
-  if (lane == 31) swarp[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int s = swarp[lane];
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, off);
-      if (lane >= off) s += y;
-    }
-    swarp[lane] = s;
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  const int ch = (c + d.nt_gu - 1) / d.nt_gu;
+  if (lane == 0) {
+    s_c[warp] = c;
+    s_ch[warp] = ch;
   }
   __syncthreads();
-  const int base = warp ? swarp[warp - 1] : 0;
-  *total = swarp[31];
-  __syncthreads();
-  return base + x - v;
-}
-
-// Counts, offsets and work lists: one CTA of 1024 threads.
-//  - counts[e] = popcount of bitmap row e; every thread takes a strided slice
-//    of the flattened [E][W] bitmap (many loads in flight) and adds into
-//    shared memory (integer adds: the result does not depend on their order);
-//  - offsets = exclusive scan of the counts;
-//  - work units of the two decode-GEMM stages, expert by expert.
-__global__ void __launch_bounds__(1024) count_scan_kernel(Dims d, Work w, int make_units) {
-  __shared__ int scount[kMaxE];
-  __shared__ int swarp[32];
-  for (int e = threadIdx.x; e < d.E; e += blockDim.x) scount[e] = 0;
-  __syncthreads();
-  const int nwords = d.E * d.W;
-  constexpr int U = 8;
-  for (int base = threadIdx.x; base < nwords; base += U * blockDim.x) {
-    unsigned m[U];
-#pragma unroll
-    for (int i = 0; i < U; ++i) {
-      const int q = base + i * blockDim.x;
-      m[i] = q < nwords ? __ldg(w.bitmap + q) : 0u;
+  if (threadIdx.x == 0) {
+    int agg_c = 0, agg_ch = 0;
+    for (int i = 0; i < 8; ++i) {
+      agg_c += s_c[i];
+      agg_ch += s_ch[i];
     }
-#pragma unroll
-    for (int i = 0; i < U; ++i) {
-      const int q = base + i * blockDim.x;
-      if (m[i]) atomicAdd(&scount[q / d.W], __popc(m[i]));
+    const int b = blockIdx.x;
+    int base_c = 0, base_ch = 0;
+    if (b == 0) {
+      st_release_u64(w.look, look_pack(2u, agg_c, agg_ch));
+    } else {
+      st_release_u64(w.look + b, look_pack(1u, agg_c, agg_ch));
+      long long t0 = 0;
+      for (int j = b - 1; j >= 0;) {
+        const unsigned long long v = ld_acquire_u64(w.look + j);
+        const unsigned state = (unsigned)(v >> 62);
+        if (state == 0u) {
+          const long long now = clock64();
+          if (t0 == 0) t0 = now;
+          else if (now - t0 > 2000000000LL) {      // ~1 s: give up, flag it
+            set_status(w.status, RL_DEV_WAIT_TIMEOUT);
+            break;
+          }
+          continue;
+        }
+        base_c += (int)(v & 0x1FFFFFFu);
+        base_ch += (int)((v >> 25) & 0xFFFFFu);
+        if (state == 2u) break;
+        --j;
+      }
+      st_release_u64(w.look + b, look_pack(2u, base_c + agg_c, base_ch + agg_ch));
     }
+    s_base_c = base_c;
+    s_base_ch = base_ch;
   }
   __syncthreads();
-
-  const int e = threadIdx.x;
-  const int c = e < d.E ? scount[e] : 0;
-  int total = 0;
-  const int off = block_excl_scan(c, swarp, &total);
-  if (e < d.E) w.offsets[e] = off;
-  if (e == 0) {
-    w.offsets[d.E] = total;
-    if (total != d.P) set_status(w.status, RL_DEV_BAD_GROUPING);
+  if (e >= d.E) return;
+  int off = s_base_c, ch0 = s_base_ch;
+  for (int i = 0; i < warp; ++i) {
+    off += s_c[i];
+    ch0 += s_ch[i];
   }
-  if (!make_units) return;
-  const int ch_gu = (c + d.nt_gu - 1) / d.nt_gu;
-  const int ch_dn = (c + d.nt_dn - 1) / d.nt_dn;
-  int tot_gu = 0, tot_dn = 0;
-  const int base_gu = block_excl_scan(ch_gu * d.slabs_gu, swarp, &tot_gu);
-  const int base_dn = block_excl_scan(ch_dn * d.groups_dn, swarp, &tot_dn);
-  const bool over = tot_gu > d.max_units_gu || tot_dn > d.max_units_dn;
-  if (e == 0) {
-    if (over) set_status(w.status, RL_DEV_UNIT_OVERFLOW);
-    w.counters[0] = over ? 0 : tot_gu;
-    w.counters[1] = over ? 0 : tot_dn;
-  }
-  if (e < d.E && !over) {
-    int q = base_gu;
-    for (int ch = 0; ch < ch_gu; ++ch) {
-      const int n0 = off + ch * d.nt_gu;
-      const int n = min(d.nt_gu, c - ch * d.nt_gu);
-      for (int s = 0; s < d.slabs_gu; ++s) w.units_gu[q++] = make_int4(e, s, n0, n);
-    }
-    q = base_dn;
-    for (int ch = 0; ch < ch_dn; ++ch) {
-      const int n0 = off + ch * d.nt_dn;
-      const int n = min(d.nt_dn, c - ch * d.nt_dn);
-      for (int s = 0; s < d.groups_dn; ++s) w.units_dn[q++] = make_int4(e, s, n0, n);
+  if (lane == 0) {
+    w.offsets[e] = off;
+    if (e == d.E - 1) {
+      const int total = off + c, tot_ch = ch0 + ch;
+      w.offsets[d.E] = total;
+      if (total != d.P) set_status(w.status, RL_DEV_BAD_GROUPING);
+      if (make_units) {
+        const bool over = tot_ch * d.slabs_gu > d.max_units_gu || tot_ch * d.groups_dn > d.max_units_dn;
+        if (over) set_status(w.status, RL_DEV_UNIT_OVERFLOW);
+        w.counters[0] = over ? 0 : tot_ch * d.slabs_gu;
+        w.counters[1] = over ? 0 : tot_ch * d.groups_dn;
+      }
     }
   }
-}
-
-// Stable scatter: one warp per expert, lanes over consecutive bitmap words;
-// pair_list[offsets[e] + r] = t*k + j for the r-th token t (ascending) that
-// chose e, and pair_pos is its inverse.  A token picks an expert at most
-// once, so ascending token is ascending pair id.
-__global__ void __launch_bounds__(256) scatter_kernel(Dims d, Work w) {
-  const int ex = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (ex >= d.E) return;
-  int running = __ldg(w.offsets + ex);
+  if (make_units) {
+    // unit q of this expert: chunk q / slabs, slab (or slab group) q % slabs
+    const int ngu = ch * d.slabs_gu, ndn = ch * d.groups_dn;
+    const int q_gu = ch0 * d.slabs_gu, q_dn = ch0 * d.groups_dn;
+    if (q_gu + ngu <= d.max_units_gu)
+      for (int u = lane; u < ngu; u += 32) {
+        const int cc = u / d.slabs_gu, sl = u - cc * d.slabs_gu;
+        w.units_gu[q_gu + u] = make_int4(e, sl, off + cc * d.nt_gu, min(d.nt_gu, c - cc * d.nt_gu));
+      }
+    if (q_dn + ndn <= d.max_units_dn)
+      for (int u = lane; u < ndn; u += 32) {
+        const int cc = u / d.groups_dn, g = u - cc * d.groups_dn;
+        w.units_dn[q_dn + u] = make_int4(e, g, off + cc * d.nt_dn, min(d.nt_dn, c - cc * d.nt_dn));
+      }
+  }
+  // stable scatter, 32 bitmap words per pass
+  int running = off;
   for (int q0 = 0; q0 < d.W; q0 += 32) {
     const int q = q0 + lane;
-    unsigned m = q < d.W ? __ldg(w.bitmap + (size_t)ex * d.W + q) : 0u;
+    unsigned m = q < d.W ? __ldg(row + q) : 0u;
     const int cnt = __popc(m);
     int incl = cnt;
 #pragma unroll
@@ -248,10 +284,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(Dims d, Work w) {
     }
     int pos = running + incl - cnt;
     while (m) {
-      const int b = __ffs(m) - 1;
+      const int bit = __ffs(m) - 1;
       m &= m - 1;
-      const int t = 32 * q + b;
-      const int j = w.jslot[(size_t)ex * d.T + t];
+      const int t = 32 * q + bit;
+      const int j = w.jslot[(size_t)e * d.T + t];
       const int pid = t * d.k + j;
       w.pair_list[pos] = pid;
       w.pair_pos[pid] = pos;
