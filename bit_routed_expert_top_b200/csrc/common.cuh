@@ -102,7 +102,7 @@ struct Work {
   unsigned long long* look;  // [ceil(E/8)] prefix records of the grouping CTAs
   int4* units_gu;        // {expert, slab, first grouped position, pairs}
   int4* units_dn;        // {expert, slab group, first grouped position, pairs}
-  __half* x16;           // [T][H] x as fp16, K-permuted per group
+  __half* x16;           // [P][H] x of the pair at each grouped position, fp16, K-permuted per group
   __half* h16;           // [P][I] h, grouped order, K-permuted per group
   __half* o16;           // [P][H] o, pair-id order
 };

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(256) gateup_simt_kernel(Dims d, Work w, Expert
       __syncthreads();
       for (int q = tid; q < 32 * kSubVals; q += blockDim.x) {
         const int i = q >> 5, v = q & 31;
-        xs[i][v] = i < nc ? __half2float(w.x16[(size_t)toks[i] * d.H + perm_pos_k<FMT>(sb * kSubVals + v)])
+        xs[i][v] = i < nc ? __half2float(w.x16[(size_t)(n0 + c0 + i) * d.H + perm_pos_k<FMT>(sb * kSubVals + v)])
                           : 0.f;
       }
       __syncthreads();

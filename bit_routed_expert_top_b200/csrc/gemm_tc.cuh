@@ -25,8 +25,8 @@
 //
 // Warp roles (24 warps, one CTA per SM, persistent over the unit list):
 //   warp 0       TMEM allocation and the single MMA-issuing thread
-//   warp 1       B operand by TMA, one elected thread: tile::gather4 of the
-//                pairs' x rows (gate/up) or a 2D tile of h rows (down), into
+//   warp 1       B operand by TMA: 2D tiles of the unit's rows of x (gate/up,
+//                gathered in grouped order beforehand) or of h (down), into
 //                the 128-byte-swizzled K-major layout
 //   warps 2..5   epilogue (one per TMEM lane quarter), double-buffered
 //                accumulators so it overlaps the next unit's MMAs
@@ -156,21 +156,13 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
-// TMA: 2D tile load and 4-row gather load into shared memory, completion
-// counted in bytes on an mbarrier (no multicast).
+// TMA: 2D tile load into shared memory, completion counted in bytes on an
+// mbarrier (no multicast).
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
           smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int y0, int y1, int y2,
-                                            int y3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4, %5, %6}], [%7];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_addr(bar))
       : "memory");
 }
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -275,7 +267,6 @@ struct Shared {
   uint64_t acc_full[kAccBufs], acc_empty[kAccBufs], drain;
   uint32_t tmem_base;
   int abort_flag;
-  int toks[kNT];
   int4 unit[kUnitCache];                 // units blockIdx.x + i*gridDim.x
   const uint8_t* blob[kUnitCache];       // their expert blobs
 };
@@ -556,43 +547,21 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     wait_bar_warp(&sh->drain, 0, sh, w.status);
   } else if (warp == 1) {
     // ------------------------------------------- B operand by TMA --------
-    // Lane 0 posts the byte count; the lanes then issue the copies in parallel
-    // (gather4: lane l takes rows 4l..4l+3); the warp stays converged.
+    // Lane 0 posts the byte count; lanes 0 and 1 each load one 64-column K
+    // block of the unit's kNT activation rows (rows past the end read zeros).
     uint32_t b_it = 0;
     bool ok = true;
     for (int ui = 0; ui < my_units && ok; ++ui) {
-      const int4 un = unit_at(ui);
-      const int cnt = un.w, n0 = un.z;
-      const int npad = max(16, (cnt + 15) & ~15);
-      if (GATEUP) {
-        // token of each pair (padding rows repeat the first pair's token)
-        __syncwarp();
-        for (int n = lane; n < npad; n += 32)
-          sh->toks[n] = w.pair_list[n0 + (n < cnt ? n : 0)] / d.k;
-        __syncwarp();
-      }
+      const int n0 = unit_at(ui).z;
       for (int kc = 0; kc < nbchunk && ok; ++kc, ++b_it) {
         const int s = b_it % kBStages;
         ok = wait_bar_warp(&sh->empty_b[s], ((b_it / kBStages) & 1) ^ 1, sh, w.status, true);
         if (!ok) break;
         uint8_t* stage = b_base + s * kBStageBytes;
-        const int rows = GATEUP ? npad : kNT;
-        if (lane == 0)
-          mbar_arrive_expect_tx(&sh->full_b[s], (uint32_t)((kBK / kBKBlock) * rows * 128));
+        if (lane == 0) mbar_arrive_expect_tx(&sh->full_b[s], (uint32_t)kBStageBytes);
         __syncwarp();
-        if (GATEUP) {
-          // lane l gathers rows 4l..4l+3 of both K blocks
-          const int n = 4 * lane;
-          if (n < npad) {
-            const int t0 = sh->toks[n], t1 = sh->toks[n + 1], t2 = sh->toks[n + 2], t3 = sh->toks[n + 3];
-#pragma unroll
-            for (int kb2 = 0; kb2 < kBK / kBKBlock; ++kb2)
-              tma_gather4(stage + kb2 * kBBlockBytes + n * 128, &bmap, kc * kBK + kb2 * kBKBlock, t0, t1, t2, t3,
-                          &sh->full_b[s]);
-          }
-        } else if (lane < kBK / kBKBlock) {
+        if (lane < kBK / kBKBlock)
           tma_load_2d(stage + lane * kBBlockBytes, &bmap, kc * kBK + lane * kBKBlock, n0, &sh->full_b[s]);
-        }
         __syncwarp();
       }
     }

@@ -39,8 +39,8 @@ constexpr int kNtGateUp = rl::tc::kNtGu;
 constexpr int kNtDown = rl::tc::kNtDn;
 constexpr int kMtDown = rl::tc::kMtDn;
 static_assert(kNtGateUp == kNtDown, "the grouping kernel derives both unit lists from one chunk prefix");
-// route, group, gate/up, down, combine
-constexpr int kLaunchesPerCall = 5;
+// route, group, x gather, gate/up, down, combine
+constexpr int kLaunchesPerCall = 6;
 
 struct Layout {
   size_t status, idx, pw, bitmap, jslot, offsets, pair_list, pair_pos, counters, look,
@@ -92,7 +92,7 @@ int plan(int fmt, int T, int H, int I, int E, int k, rl::Dims* d, Layout* L) {
   L->look = take((size_t)rl::kMaxGroupCtas * 8);
   L->units_gu = take((size_t)d->max_units_gu * 16);
   L->units_dn = take((size_t)d->max_units_dn * 16);
-  L->x16 = take((size_t)T * H * 2);
+  L->x16 = take((size_t)d->P * H * 2);
   L->h16 = take((size_t)d->P * I * 2);
   L->o16 = take((size_t)d->P * H * 2);
   L->total = o;
@@ -171,26 +171,25 @@ int make_act_map(CUtensorMap* map, const void* base, int K, long long rows, int 
 
 // Route: one CTA per 8 tokens over every byte column of the token bitmap;
 // values per lane = smallest power of two >= E/32.
-template <int FMT>
-void launch_route(const float* logits, const uint16_t* x, const rl::Dims& d, const rl::Work& w,
-                  cudaStream_t s) {
+void launch_route(const float* logits, const rl::Dims& d, const rl::Work& w, cudaStream_t s) {
   const int grid = d.W * 4;
   const int per = (d.E + 31) / 32;
-  if (per <= 1) rl::route_kernel<FMT, 1><<<grid, 256, 0, s>>>(logits, x, d, w);
-  else if (per <= 2) rl::route_kernel<FMT, 2><<<grid, 256, 0, s>>>(logits, x, d, w);
-  else if (per <= 4) rl::route_kernel<FMT, 4><<<grid, 256, 0, s>>>(logits, x, d, w);
-  else if (per <= 8) rl::route_kernel<FMT, 8><<<grid, 256, 0, s>>>(logits, x, d, w);
-  else if (per <= 16) rl::route_kernel<FMT, 16><<<grid, 256, 0, s>>>(logits, x, d, w);
-  else rl::route_kernel<FMT, 32><<<grid, 256, 0, s>>>(logits, x, d, w);
+  if (per <= 1) rl::route_kernel<1><<<grid, 256, 0, s>>>(logits, d, w);
+  else if (per <= 2) rl::route_kernel<2><<<grid, 256, 0, s>>>(logits, d, w);
+  else if (per <= 4) rl::route_kernel<4><<<grid, 256, 0, s>>>(logits, d, w);
+  else if (per <= 8) rl::route_kernel<8><<<grid, 256, 0, s>>>(logits, d, w);
+  else if (per <= 16) rl::route_kernel<16><<<grid, 256, 0, s>>>(logits, d, w);
+  else rl::route_kernel<32><<<grid, 256, 0, s>>>(logits, d, w);
 }
 
 template <int FMT>
 int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
                const rl::Work& w, float* y, cudaStream_t s) {
   mark(0, s);
-  launch_route<FMT>(logits, static_cast<const uint16_t*>(x), d, w, s);
+  launch_route(logits, d, w, s);
   mark(1, s);
   rl::group_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w, 1);
+  rl::gather_x_kernel<FMT><<<(d.P + 7) / 8, 256, 0, s>>>(static_cast<const uint16_t*>(x), d, w);
   mark(2, s);
   if (g_gemm == 1) {
     rl::gateup_simt_kernel<FMT><<<d.max_units_gu, 256, 0, s>>>(d, w, tab);
@@ -198,7 +197,7 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
     rl::down_simt_kernel<FMT><<<d.max_units_dn, 256, 0, s>>>(d, w, tab);
   } else {
     alignas(64) CUtensorMap xmap, hmap;
-    int rc = make_act_map(&xmap, w.x16, d.H, d.T, 1);
+    int rc = make_act_map(&xmap, w.x16, d.H, d.P, rl::tc::kNT);
     if (rc != RL_OK) return rc;
     rc = make_act_map(&hmap, w.h16, d.I, d.P, rl::tc::kNT);
     if (rc != RL_OK) return rc;
@@ -359,7 +358,7 @@ int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx,
   w.pair_list = pair_list;
   w.pair_pos = pair_pos;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  launch_route<RL_FMT_Q2>(router_logits, nullptr, d, w, s);
+  launch_route(router_logits, d, w, s);
   rl::group_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w, 0);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");

@@ -1,5 +1,6 @@
-// route_group.cuh - step 1 (top-k routing + softmax, plus x -> fp16) and
-// step 2 (grouping of the token/expert pairs by expert, work lists).
+// route_group.cuh - step 1 (top-k routing + softmax), step 2 (grouping of
+// the token/expert pairs by expert, work lists, x gathered in grouped order
+// as fp16) and step 5 (combine).
 //
 // "Red Lite dev72 - bounded verify, profiling", section 1: the router picks
 // each row's experts and every row keeps its own selection order; section 3:
@@ -32,11 +33,9 @@ __device__ __forceinline__ bool route_better(float v, int i, float bv, int bi) {
 //    equal value and lower expert index; -0.0 equals +0.0); only the winning
 //    lane rescans its own values.
 //  - z_j = expf(l_j - l_0) summed in j order, p_j = z_j / sum.
-//  - With x != nullptr the warp also writes its token's x row as fp16 in the
-//    K-permuted order of format FMT.
-template <int FMT, int PER>
+template <int PER>
 __global__ void __launch_bounds__(256)
-route_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ x, Dims d, Work w) {
+route_kernel(const float* __restrict__ logits, Dims d, Work w) {
   __shared__ unsigned smask[kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
@@ -100,52 +99,6 @@ route_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ x, D
     const float inv = 1.0f / sum;
     for (int j = lane; j < d.k; j += 32) w.pw[(size_t)t * d.k + j] *= inv;
 
-    if (x != nullptr) {
-      // batches of kB groups per lane: every load of a batch is issued
-      // before the first conversion
-      constexpr int G = Fmt<FMT>::kGroup;
-      constexpr int kB = 64 / G;
-      const uint16_t* xr = x + (size_t)t * d.H;
-      __half* xo = w.x16 + (size_t)t * d.H;
-      const int ng = d.H / G;
-      for (int g0 = lane; g0 < ng; g0 += kB * 32) {
-        uint4 raw[kB][G / 8];
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          const int g = g0 + u * 32;
-#pragma unroll
-          for (int q = 0; q < G / 8; ++q)
-            raw[u][q] = g < ng ? __ldg(reinterpret_cast<const uint4*>(xr + g * G) + q) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          const int g = g0 + u * 32;
-          if (g >= ng) break;
-          uint16_t in[G];
-#pragma unroll
-          for (int q = 0; q < G / 8; ++q) {
-            const uint32_t wv[4] = {raw[u][q].x, raw[u][q].y, raw[u][q].z, raw[u][q].w};
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              in[q * 8 + 2 * r] = (uint16_t)(wv[r] & 0xffffu);
-              in[q * 8 + 2 * r + 1] = (uint16_t)(wv[r] >> 16);
-            }
-          }
-          uint32_t outw[G / 2];
-#pragma unroll
-          for (int c = 0; c < G / 2; ++c) {
-            const float a = __uint_as_float((uint32_t)in[perm_value<FMT>(2 * c)] << 16);
-            const float b = __uint_as_float((uint32_t)in[perm_value<FMT>(2 * c + 1)] << 16);
-            const __half2 hh = __floats2half2_rn(a, b);
-            outw[c] = *reinterpret_cast<const uint32_t*>(&hh);
-          }
-#pragma unroll
-          for (int q = 0; q < G / 8; ++q)
-            reinterpret_cast<uint4*>(xo + g * G)[q] =
-                make_uint4(outw[4 * q], outw[4 * q + 1], outw[4 * q + 2], outw[4 * q + 3]);
-        }
-      }
-    }
   }
   __syncthreads();
   uint8_t* bm8 = reinterpret_cast<uint8_t*>(w.bitmap);
@@ -294,6 +247,62 @@ __global__ void __launch_bounds__(256) group_kernel(Dims d, Work w, int make_uni
       ++pos;
     }
     running += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+// x of every pair in grouped order, as the gate/up B operand: row pos of
+// x16 = x[t] of the pair at grouped position pos (t = pair id / k), bf16 ->
+// fp16 (exact widening to fp32, one rounding to fp16) in the K-permuted
+// order of format FMT.  One warp per grouped position.
+template <int FMT>
+__global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restrict__ x, Dims d, Work w) {
+  const int lane = threadIdx.x & 31;
+  const int pos = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (pos >= d.P) return;
+  const int t = __ldg(w.pair_list + pos) / d.k;
+  // batches of kB groups per lane: every load of a batch is issued before
+  // the first conversion
+  constexpr int G = Fmt<FMT>::kGroup;
+  constexpr int kB = 64 / G;
+  const uint16_t* xr = x + (size_t)t * d.H;
+  __half* xo = w.x16 + (size_t)pos * d.H;
+  const int ng = d.H / G;
+  for (int g0 = lane; g0 < ng; g0 += kB * 32) {
+    uint4 raw[kB][G / 8];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int g = g0 + u * 32;
+#pragma unroll
+      for (int q = 0; q < G / 8; ++q)
+        raw[u][q] = g < ng ? __ldg(reinterpret_cast<const uint4*>(xr + g * G) + q) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int g = g0 + u * 32;
+      if (g >= ng) break;
+      uint16_t in[G];
+#pragma unroll
+      for (int q = 0; q < G / 8; ++q) {
+        const uint32_t wv[4] = {raw[u][q].x, raw[u][q].y, raw[u][q].z, raw[u][q].w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          in[q * 8 + 2 * r] = (uint16_t)(wv[r] & 0xffffu);
+          in[q * 8 + 2 * r + 1] = (uint16_t)(wv[r] >> 16);
+        }
+      }
+      uint32_t outw[G / 2];
+#pragma unroll
+      for (int c = 0; c < G / 2; ++c) {
+        const float a = __uint_as_float((uint32_t)in[perm_value<FMT>(2 * c)] << 16);
+        const float b = __uint_as_float((uint32_t)in[perm_value<FMT>(2 * c + 1)] << 16);
+        const __half2 hh = __floats2half2_rn(a, b);
+        outw[c] = *reinterpret_cast<const uint32_t*>(&hh);
+      }
+#pragma unroll
+      for (int q = 0; q < G / 8; ++q)
+        reinterpret_cast<uint4*>(xo + g * G)[q] =
+            make_uint4(outw[4 * q], outw[4 * q + 1], outw[4 * q + 2], outw[4 * q + 3]);
+    }
   }
 }
 
