@@ -30,9 +30,10 @@
 //                the 128-byte-swizzled K-major layout
 //   warps 2..5   epilogue (one per TMEM lane quarter), double-buffered
 //                accumulators so it overlaps the next unit's MMAs
-//   warps 6..21  16 decoders: 4 groups = 2 M tiles x 2 sub-block parities,
-//                one warp per lane quarter; a step's A slot is handed to the
-//                MMA warp as soon as its TMEM stores have completed
+//   warps 6..21  16 decoders: 4 groups = 2 M tiles x 2 phases (the groups
+//                take the 64-value steps round-robin), one warp per TMEM lane
+//                quarter; a step's A slot is handed to the MMA warp as soon
+//                as its TMEM stores have completed
 //   warps 22,23  raw-block fetch, one warp per M tile: 16-byte cp.async of
 //                the 128 rows' blocks (consecutive lanes copy consecutive
 //                chunks of a row), completion counted on an mbarrier, up to
@@ -58,6 +59,9 @@ namespace tc {
 #ifndef RL_TC_B_STAGES
 #define RL_TC_B_STAGES 4
 #endif
+#ifndef RL_TC_DEC_PHASES
+#define RL_TC_DEC_PHASES 2
+#endif
 constexpr int kNT = RL_TC_NT;    // max pairs per unit = accumulator columns per tile
 constexpr int kNtGu = kNT;       // gate/up unit size in pairs
 constexpr int kNtDn = kNT;       // down unit size in pairs
@@ -78,8 +82,10 @@ constexpr int kBStageBytes = (kBK / kBKBlock) * kBBlockBytes;
 constexpr int kRows = kMT * 128;                // weight rows per unit
 constexpr int kEpiWarp0 = 2;
 constexpr int kDecWarp0 = 6;
-constexpr int kFetchWarp0 = 22;
-constexpr int kWarps = 24;
+constexpr int kDecPhases = RL_TC_DEC_PHASES;    // decoder groups per M tile (steps round-robin)
+constexpr int kDecWarps = 4 * kMT * kDecPhases;  // lane quarters x tiles x phases
+constexpr int kFetchWarp0 = kDecWarp0 + kDecWarps;
+constexpr int kWarps = kFetchWarp0 + kMT;
 constexpr int kThreads = kWarps * 32;
 constexpr long long kWaitCycles = 4000000000LL; // ~2 s at 2 GHz
 constexpr int kUnitCache = 64;                  // this CTA's first work units, cached in shared memory
@@ -235,6 +241,46 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 // Arrive on bar when every MMA issued so far by this warp has completed.
+// One 64-value step for both M tiles under a single elect: MMAs k = 0..3
+// (k = 2, 3 only when `full`) of tile t read A at a + 32t + 8k and B at
+// b + 2k (the descriptor address field counts 16-byte units: 16 fp16 of K
+// are 32 bytes inside a swizzled row), accumulate into d + kNT*t (overwrite
+// on `acc` = 0), then commit to `bar` (arrives when all of them have run).
+__device__ __forceinline__ void mma_step2x(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                           uint32_t full, uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t, h, eh;\n\t.reg .b32 rx, d1, a1, a2, a3, a4, a5, a6, a7;\n\t"
+      ".reg .b64 b1, b2, b3;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %4, %4;\n\t"
+      "setp.ne.b32 h, %5, 0;\n\t"
+      "and.pred eh, e, h;\n\t"
+      "add.u32 d1, %0, %7;\n\t"
+      "add.u32 a1, %1, 32;\n\t"
+      "add.u32 a2, %1, 8;\n\t"
+      "add.u32 a3, %1, 40;\n\t"
+      "add.u32 a4, %1, 16;\n\t"
+      "add.u32 a5, %1, 48;\n\t"
+      "add.u32 a6, %1, 24;\n\t"
+      "add.u32 a7, %1, 56;\n\t"
+      "add.s64 b1, %2, 2;\n\t"
+      "add.s64 b2, %2, 4;\n\t"
+      "add.s64 b3, %2, 6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [d1], [a3], b1, %3, t;\n\t"
+      "@eh tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b2, %3, t;\n\t"
+      "@eh tcgen05.mma.cta_group::1.kind::f16 [d1], [a5], b2, %3, t;\n\t"
+      "@eh tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b3, %3, t;\n\t"
+      "@eh tcgen05.mma.cta_group::1.kind::f16 [d1], [a7], b3, %3, t;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(acc), "r"(full), "r"(smem_addr(bar)), "n"(kNT)
+      : "memory");
+}
+static_assert(kSlotCols == 32, "mma_step2x addresses tile 1's A at +32 columns");
+
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
@@ -455,7 +501,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRawStages; ++s) {
       mbar_init(&sh->full_raw[s], kMT * 32); // fetch warps x 32 lanes (cp.async arrivals)
-      mbar_init(&sh->empty_raw[s], 16);      // all decoder warps
+      mbar_init(&sh->empty_raw[s], kDecWarps);  // every decoder warp releases every block
     }
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(&sh->full_b[s], 1);
@@ -495,9 +541,14 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
   if (warp == 0) {
     // ------------------------------------------------------------ MMA ---
     // The whole warp runs this loop in lockstep; one elected lane issues.
-    uint32_t ring_it = 0, b_it = 0;
+    // Ring slot / B stage indices and their phase bits advance incrementally;
+    // the loop body covers one B stage (two steps).
+    constexpr int kStepsPerB = kBK / kStepVals;
+    static_assert(kStepsPerB == 2, "one B stage = two decode steps");
+    uint32_t as = 0, aph = 0, bs = 0, bph = 0;
     bool ok = true;
     const uint64_t bdesc0 = sdesc_sw128(smem_addr(b_base));
+    const uint32_t a_base = tmem + kRingCol;
     for (int ui = 0; ui < my_units && ok; ++ui) {
       const int cnt = __shfl_sync(0xffffffffu, unit_at(ui).w, 0);
       const int npad = max(16, (cnt + 15) & ~15);
@@ -506,41 +557,26 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       if (ui >= kAccBufs) ok = wait_bar_warp(&sh->acc_empty[buf], ((ui / kAccBufs) - 1) & 1, sh, w.status);
       tc_fence_after();
       const uint32_t acc0 = tmem + buf * (kMT * kNT);
-      for (int st = 0; st < nstep && ok; ++st) {
-        constexpr int kStepsPerB = kBK / kStepVals;
-        const uint32_t bi = b_it + st / kStepsPerB;
-        const int bs = bi % kBStages;
-        if (st % kStepsPerB == 0) {
-          ok = wait_bar_warp(&sh->full_b[bs], (bi / kBStages) & 1, sh, w.status);
-          if (!ok) break;
-        }
-        const uint32_t ai = ring_it + st;
-        const int as = ai % kRing;
-        ok = wait_bar_warp(&sh->full_a[as], (ai / kRing) & 1, sh, w.status);
-        if (!ok) break;
+      for (int st = 0; st < nstep && ok; st += kStepsPerB) {
+        if (!wait_bar_warp(&sh->full_b[bs], bph, sh, w.status)) { ok = false; break; }
+        const uint64_t bd = bdesc0 + (uint64_t)((bs * kBStageBytes) >> 4);
+        // step st: K block 0 of the stage
+        if (!wait_bar_warp(&sh->full_a[as], aph, sh, w.status)) { ok = false; break; }
         tc_fence_after();
-        // B descriptor = stage base + K block of this step; +32 bytes per 16 K
-        // values inside the swizzled 128-byte rows (address field in 16 B units)
-        const uint64_t bd = bdesc0 + (uint64_t)((bs * kBStageBytes + (st % kStepsPerB) * kBBlockBytes) >> 4);
-        const uint32_t a_tm = tmem + kRingCol + as * (kMT * kSlotCols);
-        constexpr uint64_t kK16 = 32 >> 4;
-        const uint32_t first = st == 0 ? 0u : 1u;
-        mma_ts(acc0, a_tm, bd, idesc, first);
-        mma_ts(acc0 + kNT, a_tm + kSlotCols, bd, idesc, first);
-        mma_ts(acc0, a_tm + 8, bd + kK16, idesc, 1u);
-        mma_ts(acc0 + kNT, a_tm + kSlotCols + 8, bd + kK16, idesc, 1u);
-        if (2 * st + 1 < nsub) {
-          mma_ts(acc0, a_tm + 16, bd + 2 * kK16, idesc, 1u);
-          mma_ts(acc0 + kNT, a_tm + kSlotCols + 16, bd + 2 * kK16, idesc, 1u);
-          mma_ts(acc0, a_tm + 24, bd + 3 * kK16, idesc, 1u);
-          mma_ts(acc0 + kNT, a_tm + kSlotCols + 24, bd + 3 * kK16, idesc, 1u);
+        mma_step2x(acc0, a_base + as * (kMT * kSlotCols), bd, idesc, st != 0, 2 * st + 1 < nsub, &sh->empty_a[as]);
+        if (++as == kRing) { as = 0; aph ^= 1; }
+        // step st + 1: K block 1 of the stage
+        if (st + 1 < nstep) {
+          if (!wait_bar_warp(&sh->full_a[as], aph, sh, w.status)) { ok = false; break; }
+          tc_fence_after();
+          mma_step2x(acc0, a_base + as * (kMT * kSlotCols), bd + (kBBlockBytes >> 4), idesc, 1u,
+                     2 * st + 3 < nsub, &sh->empty_a[as]);
+          if (++as == kRing) { as = 0; aph ^= 1; }
         }
-        mma_commit(&sh->empty_a[as]);
-        if (st % kStepsPerB == kStepsPerB - 1 || st == nstep - 1) mma_commit(&sh->empty_b[bs]);
+        mma_commit(&sh->empty_b[bs]);
+        if (++bs == kBStages) { bs = 0; bph ^= 1; }
       }
       if (ok) mma_commit(&sh->acc_full[buf]);
-      ring_it += nstep;
-      b_it += nbchunk;
     }
     // drain: every MMA issued by this warp has completed before teardown
     mma_commit(&sh->drain);
@@ -616,9 +652,9 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     }
   } else if (warp < kFetchWarp0) {
     // ------------------------------------------------------ decoders -----
-    const int dw = warp - kDecWarp0;          // 0..15
-    const int grp = dw >> 2;                  // 0..3
-    const int tile = grp & 1, parity = grp >> 1;
+    const int dw = warp - kDecWarp0;          // 0 .. kDecWarps-1
+    const int grp = dw >> 2;                  // (tile, phase) group of four lane quarters
+    const int tile = grp % kMT, phase = grp / kMT;
     const int q = warp & 3;                   // TMEM lane quarter
     const int r = q * 32 + lane;              // lane = row inside the tile
     const uint32_t a_col = tmem + ((uint32_t)(q * 32) << 16) + kRingCol + tile * kSlotCols;
@@ -638,9 +674,9 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       rowg = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, r, gu_rowbytes, rowbytes, &R);
     };
 
-    uint32_t ring_it = 0;
+    uint32_t ring_it = 0;                     // linear index of the current unit's step 0
+    int ui = 0, kb = 0;
     for (int c = 0; c < total_blocks && ok; ++c) {
-      const int ui = c / nblk, kb = c - ui * nblk;
       row_of_unit(ui);
       const int rs = c % kRawStages;
       if (!wait_bar_warp(&sh->full_raw[rs], (c / kRawStages) & 1, sh, w.status)) { ok = false; break; }
@@ -651,8 +687,11 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       const float dd = half_bits_to_float(h0 & 0xffffu);
       const uint32_t S = (h0 >> 16) | ((h1 & 0xffu) << 16);
       const uint32_t flags = (h1 >> 8) & 0xffu;
-      // steps 4*kb .. 4*kb+3 of this block; this warp takes those of its parity
-      for (int j = parity; j < 4; j += 2) {
+      // steps 4*kb .. 4*kb+3 of this block; this warp takes those whose
+      // linear index is its phase mod kDecPhases
+      const int m = (int)((ring_it + 4u * kb) % kDecPhases);
+      const int j0 = (phase - m + kDecPhases) % kDecPhases;
+      for (int j = j0; j < 4; j += kDecPhases) {
         const int st = kb * 4 + j;
         if (2 * st >= nsub) break;
         const int i = 2 * j;                   // first sub-block of the step inside the block
@@ -695,7 +734,11 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       }
       __syncwarp();
       mbar_arrive_if(&sh->empty_raw[rs], lane == 0);
-      if (kb == nblk - 1) ring_it += nstep;
+      if (++kb == nblk) {
+        kb = 0;
+        ++ui;
+        ring_it += nstep;
+      }
     }
   } else {
     // ----------------------------------------------------- raw fetch -----
