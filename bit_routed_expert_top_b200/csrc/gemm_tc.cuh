@@ -722,10 +722,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
             !wait_bar_warp(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t dst = a_col + as * (kMT * kSlotCols);
-        tmem_st8(dst, words);
-        tmem_st8(dst + 8, words + 8);
-        tmem_st8(dst + 16, words + 16);
-        tmem_st8(dst + 24, words + 24);
+        tmem_st32(dst, words);
         // hand the slot to the MMA warp once the stores have landed
         tmem_wait_st();
         tc_fence_before();
@@ -760,14 +757,32 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
         if (!ok) break;
         uint8_t* stage = raw_base + s * raw_stage_bytes<FMT>() + tile * 128 * PITCH;
         const uint8_t* blk0 = row0 + (size_t)kb * BB;
+        if constexpr (GATEUP) {
+          // rows 552+ bytes apart: lane = row, the lane copies the 16-byte
+          // chunks that cover its row's block (fewest instructions)
+#pragma unroll
+          for (int rr0 = 0; rr0 < 128; rr0 += 32) {
+            const int rr = rr0 + lane;
+            const uintptr_t b0 = reinterpret_cast<uintptr_t>(blk0) + (uint32_t)rr * (uint32_t)rowbytes;
+            const uintptr_t a0 = b0 & ~(uintptr_t)15;
+            uint8_t* dst = stage + rr * PITCH;
+            if (rr < valid) {
+#pragma unroll
+              for (int ch = 0; ch < CHUNKS; ++ch)
+                if (a0 + 16 * ch < b0 + BB) cp_async16(dst + ch * 16, reinterpret_cast<const void*>(a0 + 16 * ch));
+            }
+          }
+        } else {
+          // short rows: consecutive lanes copy consecutive chunks of a row
 #pragma unroll 6
-        for (int i2 = 0; i2 < kCopies; ++i2) {
-          const int slot = i2 * 32 + lane;
-          const int row = slot / CHUNKS, ch = slot - row * CHUNKS;
-          const uintptr_t b0 = reinterpret_cast<uintptr_t>(blk0) + (uint32_t)row * (uint32_t)rowbytes;
-          const uintptr_t a0 = (b0 & ~(uintptr_t)15) + 16 * ch;
-          if (row < valid && a0 < b0 + BB)
-            cp_async16(stage + row * PITCH + ch * 16, reinterpret_cast<const void*>(a0));
+          for (int i2 = 0; i2 < kCopies; ++i2) {
+            const int slot = i2 * 32 + lane;
+            const int row = slot / CHUNKS, ch = slot - row * CHUNKS;
+            const uintptr_t b0 = reinterpret_cast<uintptr_t>(blk0) + (uint32_t)row * (uint32_t)rowbytes;
+            const uintptr_t a0 = (b0 & ~(uintptr_t)15) + 16 * ch;
+            if (row < valid && a0 < b0 + BB)
+              cp_async16(stage + row * PITCH + ch * 16, reinterpret_cast<const void*>(a0));
+          }
         }
         cp_async_mbar_arrive(&sh->full_raw[s]);
       }

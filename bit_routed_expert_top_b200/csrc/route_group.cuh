@@ -107,9 +107,9 @@ route_kernel(const float* __restrict__ logits, Dims d, Work w) {
     bm8[(size_t)e * row_bytes + blockIdx.x] = (uint8_t)smask[e];
 }
 
-// Prefix record of one grouping CTA, one 64-bit word: bits 0-24 pairs,
-// bits 25-44 pair chunks (units of at most nt pairs), bits 62-63 state
-// (0 nothing yet, 1 the CTA's own sums, 2 sums including every earlier CTA).
+// Record of one grouping CTA, one 64-bit word: bits 0-24 pairs, bits 25-44
+// pair chunks (units of at most nt pairs), bits 62-63 state (0 nothing yet,
+// 1 the CTA's own sums).
 __device__ __forceinline__ unsigned long long look_pack(unsigned state, int pairs, int chunks) {
   return ((unsigned long long)state << 62) | ((unsigned long long)chunks << 25) | (unsigned long long)pairs;
 }
@@ -125,10 +125,9 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
 // Step 2 in one launch of ceil(E/8) CTAs x 8 warps, warp w of CTA b owning
 // expert e = 8b + w:
 //  - count c_e = popcount of bitmap row e; chunks_e = ceil(c_e / nt);
-//  - offsets by a single-pass scan across CTAs (each CTA publishes its sums,
-//    then adds the records of the CTAs before it, walking back until one
-//    holds a full prefix; every CTA of this small grid is resident at once,
-//    and the walk is bounded);
+//  - offsets by a single-pass scan across CTAs: each CTA publishes its own
+//    sums, then adds those of every earlier CTA (read 32 at a time; every CTA
+//    of this small grid is resident at once, and the wait is bounded);
 //  - work units of both decode-GEMM stages (nt_gu == nt_dn, so both follow
 //    from the chunk prefix);
 //  - stable scatter: pair_list[offsets[e] + r] = t*k + j for the r-th token
@@ -152,40 +151,47 @@ __global__ void __launch_bounds__(256) group_kernel(Dims d, Work w, int make_uni
     s_ch[warp] = ch;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
+    // publish this CTA's sums, then add those of every earlier CTA: all of
+    // them are resident, so each publishes without waiting on another; the
+    // lanes read 32 records at a time and spin (bounded) until all are set
     int agg_c = 0, agg_ch = 0;
+#pragma unroll
     for (int i = 0; i < 8; ++i) {
       agg_c += s_c[i];
       agg_ch += s_ch[i];
     }
     const int b = blockIdx.x;
+    if (lane == 0) st_release_u64(w.look + b, look_pack(1u, agg_c, agg_ch));
     int base_c = 0, base_ch = 0;
-    if (b == 0) {
-      st_release_u64(w.look, look_pack(2u, agg_c, agg_ch));
-    } else {
-      st_release_u64(w.look + b, look_pack(1u, agg_c, agg_ch));
-      long long t0 = 0;
-      for (int j = b - 1; j >= 0;) {
-        const unsigned long long v = ld_acquire_u64(w.look + j);
-        const unsigned state = (unsigned)(v >> 62);
-        if (state == 0u) {
+    long long t0 = 0;
+    for (int j0 = 0; j0 < b; j0 += 32) {
+      const int j = j0 + lane;
+      unsigned long long v = 0;
+      if (j < b) {
+        for (;;) {
+          v = ld_acquire_u64(w.look + j);
+          if ((v >> 62) != 0u) break;
           const long long now = clock64();
           if (t0 == 0) t0 = now;
           else if (now - t0 > 2000000000LL) {      // ~1 s: give up, flag it
             set_status(w.status, RL_DEV_WAIT_TIMEOUT);
             break;
           }
-          continue;
         }
-        base_c += (int)(v & 0x1FFFFFFu);
-        base_ch += (int)((v >> 25) & 0xFFFFFu);
-        if (state == 2u) break;
-        --j;
       }
-      st_release_u64(w.look + b, look_pack(2u, base_c + agg_c, base_ch + agg_ch));
+      base_c += (int)(v & 0x1FFFFFFu);
+      base_ch += (int)((v >> 25) & 0xFFFFFu);
     }
-    s_base_c = base_c;
-    s_base_ch = base_ch;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      base_c += __shfl_xor_sync(0xffffffffu, base_c, o);
+      base_ch += __shfl_xor_sync(0xffffffffu, base_ch, o);
+    }
+    if (lane == 0) {
+      s_base_c = base_c;
+      s_base_ch = base_ch;
+    }
   }
   __syncthreads();
   if (e >= d.E) return;
