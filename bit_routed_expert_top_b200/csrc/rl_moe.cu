@@ -189,7 +189,7 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
   launch_route(logits, d, w, s);
   mark(1, s);
   rl::group_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w, 1);
-  rl::gather_x_kernel<FMT><<<(d.P + 7) / 8, 256, 0, s>>>(static_cast<const uint16_t*>(x), d, w);
+  rl::gather_x_kernel<FMT><<<(d.T + 7) / 8, 256, 0, s>>>(static_cast<const uint16_t*>(x), d, w);
   mark(2, s);
   if (g_gemm == 1) {
     rl::gateup_simt_kernel<FMT><<<d.max_units_gu, 256, 0, s>>>(d, w, tab);

@@ -257,23 +257,25 @@ __global__ void __launch_bounds__(256) group_kernel(Dims d, Work w, int make_uni
 }
 
 // x of every pair in grouped order, as the gate/up B operand: row pos of
-// x16 = x[t] of the pair at grouped position pos (t = pair id / k), bf16 ->
-// fp16 (exact widening to fp32, one rounding to fp16) in the K-permuted
-// order of format FMT.  One warp per grouped position.
+// x16 = x[t] of the pair at grouped position pos, bf16 -> fp16 (exact
+// widening to fp32, one rounding to fp16) in the K-permuted order of format
+// FMT.  One warp per token: the row is read and converted once, then stored
+// at the grouped positions of the token's k pairs (pair_pos[t*k + j]).
 template <int FMT>
 __global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restrict__ x, Dims d, Work w) {
   const int lane = threadIdx.x & 31;
-  const int pos = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (pos >= d.P) return;
-  const int t = __ldg(w.pair_list + pos) / d.k;
-  // batches of kB groups per lane: every load of a batch is issued before
-  // the first conversion
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= d.T) return;
   constexpr int G = Fmt<FMT>::kGroup;
-  constexpr int kB = 64 / G;
+  constexpr int kB = 64 / G;                 // groups per lane per batch (32 fp16 words)
   const uint16_t* xr = x + (size_t)t * d.H;
-  __half* xo = w.x16 + (size_t)pos * d.H;
   const int ng = d.H / G;
-  for (int g0 = lane; g0 < ng; g0 += kB * 32) {
+  // grouped positions of the token's pairs, lane j holding pair j (k <= 32
+  // at a time)
+  const int my_pos = lane < d.k ? __ldg(w.pair_pos + (size_t)t * d.k + lane) : 0;
+  // the batch loop is warp-uniform (the shuffles below need every lane)
+  for (int gb = 0; gb < ng; gb += kB * 32) {
+    const int g0 = gb + lane;
     uint4 raw[kB][G / 8];
 #pragma unroll
     for (int u = 0; u < kB; ++u) {
@@ -282,10 +284,9 @@ __global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restric
       for (int q = 0; q < G / 8; ++q)
         raw[u][q] = g < ng ? __ldg(reinterpret_cast<const uint4*>(xr + g * G) + q) : make_uint4(0, 0, 0, 0);
     }
+    uint4 out[kB][G / 8];
 #pragma unroll
     for (int u = 0; u < kB; ++u) {
-      const int g = g0 + u * 32;
-      if (g >= ng) break;
       uint16_t in[G];
 #pragma unroll
       for (int q = 0; q < G / 8; ++q) {
@@ -306,8 +307,19 @@ __global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restric
       }
 #pragma unroll
       for (int q = 0; q < G / 8; ++q)
-        reinterpret_cast<uint4*>(xo + g * G)[q] =
-            make_uint4(outw[4 * q], outw[4 * q + 1], outw[4 * q + 2], outw[4 * q + 3]);
+        out[u][q] = make_uint4(outw[4 * q], outw[4 * q + 1], outw[4 * q + 2], outw[4 * q + 3]);
+    }
+    for (int j = 0; j < d.k; ++j) {
+      const int pos = j < 32 ? __shfl_sync(0xffffffffu, my_pos, j) : __ldg(w.pair_pos + (size_t)t * d.k + j);
+      __half* xo = w.x16 + (size_t)pos * d.H;
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int g = g0 + u * 32;
+        if (g < ng) {
+#pragma unroll
+          for (int q = 0; q < G / 8; ++q) reinterpret_cast<uint4*>(xo + g * G)[q] = out[u][q];
+        }
+      }
     }
   }
 }
