@@ -8,7 +8,10 @@
 #pragma once
 
 #include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
 #include <cstdint>
+#include <utility>
 
 #include "../../include/rl_moe.h"
 
@@ -106,6 +109,33 @@ struct Work {
   __half* h16;           // [P][I] h, grouped order, K-permuted per group
   __half* o16;           // [P][H] o, pair-id order
 };
+
+// Programmatic dependent launch: a kernel launched with
+// cudaLaunchAttributeProgrammaticStreamSerialization may start while the
+// previous kernel of the stream is still running; pdl_wait() blocks until
+// that kernel has completed and its writes are visible (a no-op without
+// such a predecessor), and pdl_trigger() lets the next kernel start early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch `kernel` on `s`, overlapping its start with the previous kernel of
+// the stream when `pdl` (the kernel must call pdl_wait() before it reads
+// anything that kernel wrote).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            bool pdl, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 __device__ __forceinline__ void set_status(unsigned* st, unsigned bits) {
   atomicOr(st, bits);

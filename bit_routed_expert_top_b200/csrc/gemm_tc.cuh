@@ -465,6 +465,8 @@ __device__ __forceinline__ const uint8_t* tile_row(const Dims& d, const uint8_t*
 template <int FMT, bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUtensorMap bmap) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* raw_base = smem_raw;
   uint8_t* b_base = raw_base + kRawStages * raw_stage_bytes<FMT>();
@@ -606,12 +608,20 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    static_assert(kNT <= 64, "the down epilogue keeps two pair ids per lane");
     for (int ui = 0; ui < my_units; ++ui) {
       const int4 un = unit_at(ui);
       const int buf = ui & 1;
+      const int cnt = un.w, n0 = un.z;
+      // down: the unit's pair ids (o rows), lane l holding pairs l and 32 + l,
+      // loaded before the wait
+      int pid_lo = 0, pid_hi = 0;
+      if (!GATEUP) {
+        if (lane < cnt) pid_lo = __ldg(w.pair_list + n0 + lane);
+        if (32 + lane < cnt) pid_hi = __ldg(w.pair_list + n0 + 32 + lane);
+      }
       if (!wait_bar_warp(&sh->acc_full[buf], (ui / kAccBufs) & 1, sh, w.status, true)) break;
       tc_fence_after();
-      const int cnt = un.w, n0 = un.z;
       const uint32_t acc0 = tmem + lane_addr + buf * (kMT * kNT);
       for (int cc = 0; cc * 16 < cnt; ++cc) {
         uint32_t a0[16], a1[16];
@@ -638,8 +648,8 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = cc * 16 + j;
+            const int pid = __shfl_sync(0xffffffffu, n < 32 ? pid_lo : pid_hi, n & 31);
             if (n < cnt) {
-              const int pid = __ldg(w.pair_list + n0 + n);
               if (r0 < d.H) w.o16[(size_t)pid * d.H + r0] = __float2half_rn(__uint_as_float(a0[j]));
               if (r1 < d.H) w.o16[(size_t)pid * d.H + r1] = __float2half_rn(__uint_as_float(a1[j]));
             }
@@ -810,7 +820,8 @@ inline int num_sms() {
 }
 
 template <int FMT, bool GATEUP>
-int launch(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& bmap, cudaStream_t s) {
+int launch(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& bmap, cudaStream_t s,
+           bool pdl) {
   static bool configured = false;
   constexpr int smem = smem_bytes<FMT>();
   if (!configured) {
@@ -821,17 +832,21 @@ int launch(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorM
   }
   const int maxu = GATEUP ? d.max_units_gu : d.max_units_dn;
   const int grid = maxu < num_sms() ? maxu : num_sms();
-  decode_gemm_kernel<FMT, GATEUP><<<grid, kThreads, smem, s>>>(d, w, tab, bmap);
-  return RL_OK;
+  return launch_k(decode_gemm_kernel<FMT, GATEUP>, dim3(grid), dim3(kThreads), smem, s, pdl, d, w, tab, bmap) ==
+                 cudaSuccess
+             ? RL_OK
+             : RL_ERR_CUDA;
 }
 
 template <int FMT>
-int launch_gateup(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& xmap, cudaStream_t s) {
-  return launch<FMT, true>(d, w, tab, xmap, s);
+int launch_gateup(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& xmap, cudaStream_t s,
+                  bool pdl) {
+  return launch<FMT, true>(d, w, tab, xmap, s, pdl);
 }
 template <int FMT>
-int launch_down(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& hmap, cudaStream_t s) {
-  return launch<FMT, false>(d, w, tab, hmap, s);
+int launch_down(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& hmap, cudaStream_t s,
+                bool pdl) {
+  return launch<FMT, false>(d, w, tab, hmap, s, pdl);
 }
 
 }  // namespace tc

@@ -186,10 +186,14 @@ template <int FMT>
 int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
                const rl::Work& w, float* y, cudaStream_t s) {
   mark(0, s);
+  // kernels after the first start while their predecessor drains
+  // (programmatic dependent launch), except when stage events sit between
+  const bool pdl = !g_prof;
   launch_route(logits, d, w, s);
   mark(1, s);
-  rl::group_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w, 1);
-  rl::gather_x_kernel<FMT><<<(d.T + 7) / 8, 256, 0, s>>>(static_cast<const uint16_t*>(x), d, w);
+  rl::launch_k(rl::group_kernel, dim3((d.E + 7) / 8), dim3(256), 0, s, pdl, d, w, 1);
+  rl::launch_k(rl::gather_x_kernel<FMT>, dim3((d.T + 7) / 8), dim3(256), 0, s, pdl,
+               static_cast<const uint16_t*>(x), d, w);
   mark(2, s);
   if (g_gemm == 1) {
     rl::gateup_simt_kernel<FMT><<<d.max_units_gu, 256, 0, s>>>(d, w, tab);
@@ -201,14 +205,15 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
     if (rc != RL_OK) return rc;
     rc = make_act_map(&hmap, w.h16, d.I, d.P, rl::tc::kNT);
     if (rc != RL_OK) return rc;
-    rc = rl::tc::launch_gateup<FMT>(d, w, tab, xmap, s);
+    rc = rl::tc::launch_gateup<FMT>(d, w, tab, xmap, s, pdl);
     if (rc != RL_OK) return rc;
     mark(3, s);
-    rc = rl::tc::launch_down<FMT>(d, w, tab, hmap, s);
+    rc = rl::tc::launch_down<FMT>(d, w, tab, hmap, s, pdl);
     if (rc != RL_OK) return rc;
   }
   mark(4, s);
-  rl::combine_kernel<<<dim3(d.T, (d.H + 1023) / 1024), 128, 0, s>>>(d, w.pw, w.o16, y);
+  rl::launch_k(rl::combine_kernel, dim3(d.T, (d.H + 1023) / 1024), dim3(128), 0, s, pdl,
+               d, static_cast<const float*>(w.pw), static_cast<const __half*>(w.o16), y);
   mark(5, s);
   if (g_prof) g_ev_recorded = true;
   const cudaError_t e = cudaGetLastError();

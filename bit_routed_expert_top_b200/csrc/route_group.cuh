@@ -36,6 +36,7 @@ __device__ __forceinline__ bool route_better(float v, int i, float bv, int bi) {
 template <int PER>
 __global__ void __launch_bounds__(256)
 route_kernel(const float* __restrict__ logits, Dims d, Work w) {
+  pdl_trigger();
   __shared__ unsigned smask[kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
@@ -135,6 +136,8 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
 //    an expert at most once, so ascending token is ascending pair id.
 // The route kernel zeroes the prefix records before this kernel runs.
 __global__ void __launch_bounds__(256) group_kernel(Dims d, Work w, int make_units) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_c[8], s_ch[8];
   __shared__ int s_base_c, s_base_ch;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -263,6 +266,8 @@ __global__ void __launch_bounds__(256) group_kernel(Dims d, Work w, int make_uni
 // at the grouped positions of the token's k pairs (pair_pos[t*k + j]).
 template <int FMT>
 __global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restrict__ x, Dims d, Work w) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= d.T) return;
@@ -330,6 +335,8 @@ __global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restric
 __global__ void __launch_bounds__(256)
 combine_kernel(Dims d, const float* __restrict__ pw, const __half* __restrict__ o16,
                float* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
   if (c >= d.H) return;
