@@ -9,7 +9,9 @@ the library's C ABI (rl_moe_prefill_ws).  Default workload: the 2,048-token
 chunk, H=2048, I=512, 512 experts, top-10, format Q2 (20,480 pairs).  The L2
 is flushed (a 256 MB device write) before every timed step; each step is timed
 with CUDA events on the launching stream.  The metric is routed pairs/s (the
-layer's ms per step is in ms_per_step).
+layer's ms per step is in ms_per_step).  A second timed pass records the
+library's CUDA events between its kernels for the stage times and the gate/up
+kernel's duration (the roofline figure).
 
 Multi-GPU: the layer does not shard (one GPU per layer call), so --gpus N runs
 N independent replicas, one process per GPU under torchrun; value is the pairs
