@@ -135,6 +135,24 @@ class ClockSampler:
                 "samples": len(self.rows)}
 
 
+def max_over_ranks(x, world, device=None):
+    """Max of a per-rank number over all ranks (every rank calls it at the
+    same point, so it is also how an error on one rank reaches the others)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world, steps, units_per_step, max_ms):
+    """Whole-job units/s of `world` replicas, each doing `units_per_step`
+    per step, timed by the slowest rank's total over `steps` steps."""
+    return world * steps * units_per_step / (max_ms * 1e-3)
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -218,7 +236,8 @@ def bench_ours(args, wl, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", device_id=dev)
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
 
     inp = synth.make_inputs(wl)
     x = torch.from_numpy(inp.x_bits.view(np.int16).copy()).to(dev)
@@ -239,8 +258,8 @@ def bench_ours(args, wl, world, rank, local):
         layer()
     torch.cuda.synchronize()
     bits = api.rl_moe_check_status(ws, stream)
-    if bits:
-        raise SystemExit(f"device status 0x{bits:x}: {api.rl_last_error()}")
+    if max_over_ranks(bits, world, dev):
+        raise SystemExit(f"device status 0x{bits:x} on rank {rank}: {api.rl_last_error()}")
 
     # touched experts (for the byte count of the roofline)
     idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
@@ -283,14 +302,10 @@ def bench_ours(args, wl, world, rank, local):
     clocks = sampler.stop()
     api.rl_moe_profile_enable(False)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     bits = api.rl_moe_check_status(ws, stream)
-    if bits:
-        raise SystemExit(f"device status 0x{bits:x}: {api.rl_last_error()}")
+    if max_over_ranks(bits, world, dev):
+        raise SystemExit(f"device status 0x{bits:x} on rank {rank}: {api.rl_last_error()}")
 
     # end to end: pinned host inputs and output, copies inside the timed region
     hx = torch.from_numpy(inp.x_bits.view(np.int16).copy()).pin_memory()
@@ -309,11 +324,8 @@ def bench_ours(args, wl, world, rank, local):
         if i >= args.warmup:
             e_ends[i - args.warmup].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), world, dev)
     if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
@@ -329,7 +341,7 @@ def bench_ours(args, wl, world, rank, local):
                     model["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
     kernel_file = os.path.join(ROOT, "bit_routed_expert_top_b200", "csrc", "gemm_tc.cuh")
     traffic = read_traffic(kernel_file)
-    value = world * args.steps * P / (total_ms * 1e-3)
+    value = replica_throughput(world, args.steps, P, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -349,7 +361,7 @@ def bench_ours(args, wl, world, rank, local):
                            "algorithmic_bytes": model["bytes"]},
         "stages_ms": {k: statistics.mean(s[k] for s in stage_ms) for k in stage_ms[0]},
         "routed_tokens_per_s": world * args.steps * wl.T / (total_ms * 1e-3),
-        "e2e": {"value": world * args.steps * P / (e2e_ms * 1e-3), "unit": UNIT,
+        "e2e": {"value": replica_throughput(world, args.steps, P, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * 2 + logits.numel() * 4),
                 "d2h_bytes_per_step": int(y.numel() * 4)},
         "gpu_launches": args.steps * api.rl_moe_launches_per_call(),
