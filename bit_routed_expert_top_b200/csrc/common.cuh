@@ -97,7 +97,7 @@ struct Work {
   int* idx;              // [P] expert of pair t*k+j
   float* pw;             // [P] routing weight p_{t,j}
   unsigned* bitmap;      // [E][W] bit b of word w: token 32w+b chose expert e
-  uint16_t* jslot;       // [E][T] slot j of token t for expert e (valid where bit set)
+  int* wprefix;          // [E][W] grouped position of the first pair of expert e in bitmap word w
   int* offsets;          // [E+1]
   int* pair_list;        // [P] grouped by expert, ascending token
   int* pair_pos;         // [P] inverse

@@ -39,11 +39,11 @@ constexpr int kNtGateUp = rl::tc::kNtGu;
 constexpr int kNtDown = rl::tc::kNtDn;
 constexpr int kMtDown = rl::tc::kMtDn;
 static_assert(kNtGateUp == kNtDown, "the grouping kernel derives both unit lists from one chunk prefix");
-// route, group, x gather, gate/up, down, combine
+// route, group, pair placement + x gather, gate/up, down, combine
 constexpr int kLaunchesPerCall = 6;
 
 struct Layout {
-  size_t status, idx, pw, bitmap, jslot, offsets, pair_list, pair_pos, counters, look,
+  size_t status, idx, pw, bitmap, wprefix, offsets, pair_list, pair_pos, counters, look,
       units_gu, units_dn, x16, h16, o16, total;
 };
 
@@ -84,7 +84,7 @@ int plan(int fmt, int T, int H, int I, int E, int k, rl::Dims* d, Layout* L) {
   L->idx = take((size_t)d->P * 4);
   L->pw = take((size_t)d->P * 4);
   L->bitmap = take((size_t)E * d->W * 4);
-  L->jslot = take((size_t)E * T * 2);
+  L->wprefix = take((size_t)E * d->W * 4);
   L->offsets = take((size_t)(E + 1) * 4);
   L->pair_list = take((size_t)d->P * 4);
   L->pair_pos = take((size_t)d->P * 4);
@@ -106,7 +106,7 @@ rl::Work carve(void* ws, const Layout& L) {
   w.idx = reinterpret_cast<int*>(b + L.idx);
   w.pw = reinterpret_cast<float*>(b + L.pw);
   w.bitmap = reinterpret_cast<unsigned*>(b + L.bitmap);
-  w.jslot = reinterpret_cast<uint16_t*>(b + L.jslot);
+  w.wprefix = reinterpret_cast<int*>(b + L.wprefix);
   w.offsets = reinterpret_cast<int*>(b + L.offsets);
   w.pair_list = reinterpret_cast<int*>(b + L.pair_list);
   w.pair_pos = reinterpret_cast<int*>(b + L.pair_pos);
@@ -192,7 +192,7 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
   launch_route(logits, d, w, s);
   mark(1, s);
   rl::launch_k(rl::group_kernel, dim3((d.E + 7) / 8), dim3(256), 0, s, pdl, d, w, 1);
-  rl::launch_k(rl::gather_x_kernel<FMT>, dim3((d.T + 7) / 8), dim3(256), 0, s, pdl,
+  rl::launch_k(rl::place_pairs_kernel<FMT>, dim3((d.T + 7) / 8), dim3(256), 0, s, pdl,
                static_cast<const uint16_t*>(x), d, w);
   mark(2, s);
   if (g_gemm == 1) {
@@ -365,6 +365,7 @@ int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   launch_route(router_logits, d, w, s);
   rl::group_kernel<<<(d.E + 7) / 8, 256, 0, s>>>(d, w, 0);
+  rl::place_pairs_kernel<RL_FMT_Q2><<<(d.T + 7) / 8, 256, 0, s>>>(nullptr, d, w);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return RL_OK;

@@ -15,12 +15,12 @@
 
 namespace rl {
 
-// (value, index) "better" = larger value, or equal value (IEEE ==, so -0.0
-// equals +0.0) and lower index.  idx < 0 marks "nothing".
-__device__ __forceinline__ bool route_better(float v, int i, float bv, int bi) {
-  if (i < 0) return false;
-  if (bi < 0) return true;
-  return v > bv || (v == bv && i < bi);
+// Order-preserving map of a finite fp32 to u32 (larger value -> larger key;
+// -0.0 is mapped as +0.0, so equal values get equal keys).  Key 0 is never
+// produced by a finite value and marks "nothing".
+__device__ __forceinline__ unsigned route_key(float v) {
+  const unsigned u = __float_as_uint(v == 0.0f ? 0.0f : v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 // One CTA of 8 warps handles 8 consecutive tokens (one byte column of the
@@ -73,14 +73,12 @@ route_kernel(const float* __restrict__ logits, Dims d, Work w) {
     rescan(mv, mi);
     float l0 = 0.f, sum = 0.f;
     for (int j = 0; j < d.k; ++j) {
-      float bv = mv;
-      int bi = mi;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (route_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-      }
+      // warp-wide best of the lanes' bests: the largest key, then among the
+      // lanes holding it the lowest expert index (two warp reductions)
+      const unsigned key = mi < 0 ? 0u : route_key(mv);
+      const unsigned kmax = __reduce_max_sync(0xffffffffu, key);
+      const int bi = (int)__reduce_min_sync(0xffffffffu, key == kmax && mi >= 0 ? (unsigned)mi : 0xFFFFFFFFu);
+      const float bv = __shfl_sync(0xffffffffu, mv, bi & 31);
       if ((bi & 31) == lane) {
         taken |= 1u << (bi >> 5);
         rescan(mv, mi);
@@ -92,10 +90,7 @@ route_kernel(const float* __restrict__ logits, Dims d, Work w) {
         w.idx[(size_t)t * d.k + j] = bi;
         w.pw[(size_t)t * d.k + j] = z;
       }
-      if (lane == 0) {
-        atomicOr(&smask[bi], 1u << warp);
-        if (w.jslot) w.jslot[(size_t)bi * d.T + t] = (uint16_t)j;
-      }
+      if (lane == 0) atomicOr(&smask[bi], 1u << warp);
     }
     const float inv = 1.0f / sum;
     for (int j = lane; j < d.k; j += 32) w.pw[(size_t)t * d.k + j] *= inv;
@@ -131,9 +126,8 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
 //    of this small grid is resident at once, and the wait is bounded);
 //  - work units of both decode-GEMM stages (nt_gu == nt_dn, so both follow
 //    from the chunk prefix);
-//  - stable scatter: pair_list[offsets[e] + r] = t*k + j for the r-th token
-//    t (ascending) that chose e, and pair_pos is its inverse.  A token picks
-//    an expert at most once, so ascending token is ascending pair id.
+//  - per bitmap word, the grouped position of the expert's first pair in it
+//    (wprefix), from which place_pairs_kernel puts each pair in place.
 // The route kernel zeroes the prefix records before this kernel runs.
 __global__ void __launch_bounds__(256) group_kernel(Dims d, Work w, int make_units) {
   pdl_wait();
@@ -232,52 +226,60 @@ __global__ void __launch_bounds__(256) group_kernel(Dims d, Work w, int make_uni
         w.units_dn[q_dn + u] = make_int4(e, g, off + cc * d.nt_dn, min(d.nt_dn, c - cc * d.nt_dn));
       }
   }
-  // stable scatter, 32 bitmap words per pass
+  // grouped position of the expert's first pair in each bitmap word (the
+  // pairs themselves are placed per token by place_pairs_kernel)
   int running = off;
   for (int q0 = 0; q0 < d.W; q0 += 32) {
     const int q = q0 + lane;
-    unsigned m = q < d.W ? __ldg(row + q) : 0u;
-    const int cnt = __popc(m);
+    const int cnt = q < d.W ? __popc(__ldg(row + q)) : 0;
     int incl = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    int pos = running + incl - cnt;
-    while (m) {
-      const int bit = __ffs(m) - 1;
-      m &= m - 1;
-      const int t = 32 * q + bit;
-      const int j = w.jslot[(size_t)e * d.T + t];
-      const int pid = t * d.k + j;
-      w.pair_list[pos] = pid;
-      w.pair_pos[pid] = pos;
-      ++pos;
-    }
+    if (q < d.W) w.wprefix[(size_t)e * d.W + q] = running + incl - cnt;
     running += __shfl_sync(0xffffffffu, incl, 31);
   }
 }
 
-// x of every pair in grouped order, as the gate/up B operand: row pos of
-// x16 = x[t] of the pair at grouped position pos, bf16 -> fp16 (exact
-// widening to fp32, one rounding to fp16) in the K-permuted order of format
-// FMT.  One warp per token: the row is read and converted once, then stored
-// at the grouped positions of the token's k pairs (pair_pos[t*k + j]).
+// Stable scatter and x gather, one warp per token t:
+//  - pair t*k + j (expert e = idx[t*k+j]) goes to grouped position
+//    wprefix[e][t/32] + (number of tokens below t in word t/32 that chose e),
+//    i.e. pair_list[offsets[e] + r] = t*k + j for the r-th token t
+//    (ascending) that chose e; pair_pos is the inverse.  A token picks an
+//    expert at most once, so ascending token is ascending pair id;
+//  - with x != nullptr, row pos of x16 = x[t] for each of the token's pairs,
+//    bf16 -> fp16 (exact widening to fp32, one rounding to fp16) in the
+//    K-permuted order of format FMT: the row is read and converted once.
 template <int FMT>
-__global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restrict__ x, Dims d, Work w) {
+__global__ void __launch_bounds__(256) place_pairs_kernel(const uint16_t* __restrict__ x, Dims d, Work w) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= d.T) return;
+  const int wq = t >> 5;
+  const unsigned below = (1u << (t & 31)) - 1u;
+  int my_pos = 0;                            // position of pair j = lane (j < 32)
+  for (int j0 = 0; j0 < d.k; j0 += 32) {
+    const int j = j0 + lane;
+    if (j < d.k) {
+      const int pid = t * d.k + j;
+      const int e = __ldg(w.idx + pid);
+      const size_t wi = (size_t)e * d.W + wq;
+      const int pos = __ldg(w.wprefix + wi) + __popc(__ldg(w.bitmap + wi) & below);
+      w.pair_list[pos] = pid;
+      w.pair_pos[pid] = pos;
+      if (j0 == 0) my_pos = pos;
+    }
+  }
+  if (x == nullptr) return;
+  __syncwarp();                              // pair_pos of j >= 32 is read back below
   constexpr int G = Fmt<FMT>::kGroup;
   constexpr int kB = 64 / G;                 // groups per lane per batch (32 fp16 words)
   const uint16_t* xr = x + (size_t)t * d.H;
   const int ng = d.H / G;
-  // grouped positions of the token's pairs, lane j holding pair j (k <= 32
-  // at a time)
-  const int my_pos = lane < d.k ? __ldg(w.pair_pos + (size_t)t * d.k + lane) : 0;
   // the batch loop is warp-uniform (the shuffles below need every lane)
   for (int gb = 0; gb < ng; gb += kB * 32) {
     const int g0 = gb + lane;
@@ -315,7 +317,7 @@ __global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restric
         out[u][q] = make_uint4(outw[4 * q], outw[4 * q + 1], outw[4 * q + 2], outw[4 * q + 3]);
     }
     for (int j = 0; j < d.k; ++j) {
-      const int pos = j < 32 ? __shfl_sync(0xffffffffu, my_pos, j) : __ldg(w.pair_pos + (size_t)t * d.k + j);
+      const int pos = j < 32 ? __shfl_sync(0xffffffffu, my_pos, j) : w.pair_pos[(size_t)t * d.k + j];
       __half* xo = w.x16 + (size_t)pos * d.H;
 #pragma unroll
       for (int u = 0; u < kB; ++u) {
