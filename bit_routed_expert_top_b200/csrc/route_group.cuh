@@ -33,6 +33,60 @@ __device__ __forceinline__ unsigned route_key(float v) {
 //    equal value and lower expert index; -0.0 equals +0.0); only the winning
 //    lane rescans its own values.
 //  - z_j = expf(l_j - l_0) summed in j order, p_j = z_j / sum.
+// Top-k of one token's logits row by one warp (see route_kernel): writes
+// idx[j] and the normalised p[j] for j = 0..k-1 in selection order and calls
+// on_pick(expert) on lane 0 for every pick.
+template <int PER, typename OnPick>
+__device__ __forceinline__ void route_token(const float* __restrict__ row, int E, int k, int lane, int* idx,
+                                            float* pw, OnPick on_pick) {
+  float v[PER];
+  unsigned taken = 0u;
+#pragma unroll
+  for (int m = 0; m < PER; ++m) {
+    const int e = lane + 32 * m;
+    if (e < E) v[m] = __ldg(row + e);
+    else { v[m] = 0.f; taken |= 1u << m; }
+  }
+  // this lane's best untaken entry
+  auto rescan = [&](float& bv, int& bi) {
+    bv = 0.f;
+    bi = -1;
+#pragma unroll
+    for (int m = 0; m < PER; ++m) {
+      const bool free_m = !((taken >> m) & 1u);
+      // strict '>' keeps the lower index on equal values (m ascending)
+      if (free_m && (bi < 0 || v[m] > bv)) { bv = v[m]; bi = lane + 32 * m; }
+    }
+  };
+  float mv;
+  int mi;
+  rescan(mv, mi);
+  float l0 = 0.f, sum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    // warp-wide best of the lanes' bests: the largest key, then among the
+    // lanes holding it the lowest expert index (two warp reductions)
+    const unsigned key = mi < 0 ? 0u : route_key(mv);
+    const unsigned kmax = __reduce_max_sync(0xffffffffu, key);
+    const int bi = (int)__reduce_min_sync(0xffffffffu, key == kmax && mi >= 0 ? (unsigned)mi : 0xFFFFFFFFu);
+    const float bv = __shfl_sync(0xffffffffu, mv, bi & 31);
+    if ((bi & 31) == lane) {
+      taken |= 1u << (bi >> 5);
+      rescan(mv, mi);
+    }
+    if (j == 0) l0 = bv;
+    const float z = expf(bv - l0);
+    sum += z;                                   // same value in every lane
+    if ((j & 31) == lane) {
+      idx[j] = bi;
+      pw[j] = z;
+    }
+    if (lane == 0) on_pick(bi);
+  }
+  const float inv = 1.0f / sum;
+  __syncwarp();
+  for (int j = lane; j < k; j += 32) pw[j] *= inv;
+}
+
 template <int PER>
 __global__ void __launch_bounds__(256)
 route_kernel(const float* __restrict__ logits, Dims d, Work w) {
@@ -46,56 +100,9 @@ route_kernel(const float* __restrict__ logits, Dims d, Work w) {
   }
   for (int e = threadIdx.x; e < d.E; e += blockDim.x) smask[e] = 0u;
   __syncthreads();
-
-  if (t < d.T) {
-    const float* row = logits + (size_t)t * d.E;
-    float v[PER];
-    unsigned taken = 0u;
-#pragma unroll
-    for (int m = 0; m < PER; ++m) {
-      const int e = lane + 32 * m;
-      if (e < d.E) v[m] = __ldg(row + e);
-      else { v[m] = 0.f; taken |= 1u << m; }
-    }
-    // this lane's best untaken entry
-    auto rescan = [&](float& bv, int& bi) {
-      bv = 0.f;
-      bi = -1;
-#pragma unroll
-      for (int m = 0; m < PER; ++m) {
-        const bool free_m = !((taken >> m) & 1u);
-        // strict '>' keeps the lower index on equal values (m ascending)
-        if (free_m && (bi < 0 || v[m] > bv)) { bv = v[m]; bi = lane + 32 * m; }
-      }
-    };
-    float mv;
-    int mi;
-    rescan(mv, mi);
-    float l0 = 0.f, sum = 0.f;
-    for (int j = 0; j < d.k; ++j) {
-      // warp-wide best of the lanes' bests: the largest key, then among the
-      // lanes holding it the lowest expert index (two warp reductions)
-      const unsigned key = mi < 0 ? 0u : route_key(mv);
-      const unsigned kmax = __reduce_max_sync(0xffffffffu, key);
-      const int bi = (int)__reduce_min_sync(0xffffffffu, key == kmax && mi >= 0 ? (unsigned)mi : 0xFFFFFFFFu);
-      const float bv = __shfl_sync(0xffffffffu, mv, bi & 31);
-      if ((bi & 31) == lane) {
-        taken |= 1u << (bi >> 5);
-        rescan(mv, mi);
-      }
-      if (j == 0) l0 = bv;
-      const float z = expf(bv - l0);
-      sum += z;                                   // same value in every lane
-      if ((j & 31) == lane) {
-        w.idx[(size_t)t * d.k + j] = bi;
-        w.pw[(size_t)t * d.k + j] = z;
-      }
-      if (lane == 0) atomicOr(&smask[bi], 1u << warp);
-    }
-    const float inv = 1.0f / sum;
-    for (int j = lane; j < d.k; j += 32) w.pw[(size_t)t * d.k + j] *= inv;
-
-  }
+  if (t < d.T)
+    route_token<PER>(logits + (size_t)t * d.E, d.E, d.k, lane, w.idx + (size_t)t * d.k, w.pw + (size_t)t * d.k,
+                     [&](int e) { atomicOr(&smask[e], 1u << warp); });
   __syncthreads();
   uint8_t* bm8 = reinterpret_cast<uint8_t*>(w.bitmap);
   const size_t row_bytes = (size_t)d.W * 4;

@@ -120,6 +120,22 @@ def test_layer_small_every_output(wl):
     Hh.assert_y_close(y, ref["y"], wl.name)
 
 
+@pytest.mark.parametrize("wl", [
+    synth.WORKLOADS[1],                                             # verify2: T=2, 512 experts, top-10
+    synth.Workload("st_t3_q1", 3, 352, 96, 7, 2, synth.FMT_Q1),     # ragged K, Q1
+    synth.Workload("st_t6", 6, 256, 128, 64, 10, synth.FMT_Q2),     # P = 60
+    synth.Workload("st_t64_k1", 64, 256, 128, 8, 1, synth.FMT_Q1),  # P = 64, the largest on this path
+    synth.Workload("st_e1024", 2, 512, 256, 1024, 8, synth.FMT_Q2), # 32 logits per lane
+], ids=lambda w: w.name)
+def test_small_chunks_every_output(wl):
+    """Chunks of at most 64 pairs (decode / verify steps): every output
+    against the oracle."""
+    inp = synth.make_inputs(wl, seed=7 + sum(wl.name.encode()))
+    y, _ = run_prefill(inp)
+    ref = full_oracle(inp)
+    Hh.assert_y_close(y, ref["y"], wl.name)
+
+
 def test_layer_heavy_expert_many_n_tiles():
     """One expert takes every token (n_e = T > one N tile), most experts
     get no pair at all."""
