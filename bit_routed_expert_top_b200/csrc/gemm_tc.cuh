@@ -35,9 +35,10 @@
 //                quarter; a step's A slot is handed to the MMA warp as soon
 //                as its TMEM stores have completed
 //   warps 22,23  raw-block fetch, one warp per M tile: 16-byte cp.async of
-//                the 128 rows' blocks (consecutive lanes copy consecutive
-//                chunks of a row), completion counted on an mbarrier, up to
-//                kRawStages K blocks ahead of the decoders
+//                the 128 rows' blocks (gate/up: one lane per row; down:
+//                consecutive lanes on consecutive chunks of a row),
+//                completion counted on an mbarrier, up to kRawStages K blocks
+//                ahead of the decoders
 // Every wait is bounded: on timeout the CTA raises RL_DEV_WAIT_TIMEOUT in
 // the status word and all roles leave their loops.
 #pragma once
@@ -155,13 +156,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
 // TMA: 2D tile load into shared memory, completion counted in bytes on an
 // mbarrier (no multicast).
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -174,33 +168,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-      : "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
@@ -226,21 +198,10 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// D[tmem] (+)= A[tmem] * B[smem], fp16 x fp16 -> fp32, cta_group::1.  Called
-// by a whole converged warp with warp-uniform operands; one elected lane
-// issues (operands then live in uniform registers: issuing from a divergent
+// D[tmem] (+)= A[tmem] * B[smem], fp16 x fp16 -> fp32, cta_group::1, issued
+// by a whole converged warp with warp-uniform operands through one elected
+// lane (operands then live in uniform registers: issuing from a divergent
 // single lane measured ~2x slower per instruction).
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b32 rx;\n\t"
-      "elect.sync rx|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Arrive on bar when every MMA issued so far by this warp has completed.
 // One 64-value step for both M tiles under a single elect: MMAs k = 0..3
 // (k = 2, 3 only when `full`) of tile t read A at a + 32t + 8k and B at
 // b + 2k (the descriptor address field counts 16-byte units: 16 fp16 of K
@@ -281,6 +242,7 @@ __device__ __forceinline__ void mma_step2x(uint32_t d, uint32_t a, uint64_t b, u
 }
 static_assert(kSlotCols == 32, "mma_step2x addresses tile 1's A at +32 columns");
 
+// Arrive on bar when every MMA issued so far by this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
