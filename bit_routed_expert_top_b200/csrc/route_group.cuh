@@ -285,6 +285,10 @@ __global__ void __launch_bounds__(256) place_pairs_kernel(const uint16_t* __rest
   __syncwarp();                              // pair_pos of j >= 32 is read back below
   constexpr int G = Fmt<FMT>::kGroup;
   constexpr int kB = 64 / G;                 // groups per lane per batch (32 fp16 words)
+  // a batch (2,048 values) is converted once into this warp's shared-memory
+  // buffer, then written to the k rows by bulk asynchronous copies
+  __shared__ __align__(128) uint4 stage_all[8][kB * 32 * G / 8];
+  uint4* stage = stage_all[threadIdx.x >> 5];
   const uint16_t* xr = x + (size_t)t * d.H;
   const int ng = d.H / G;
   // the batch loop is warp-uniform (the shuffles below need every lane)
@@ -323,19 +327,34 @@ __global__ void __launch_bounds__(256) place_pairs_kernel(const uint16_t* __rest
       for (int q = 0; q < G / 8; ++q)
         out[u][q] = make_uint4(outw[4 * q], outw[4 * q + 1], outw[4 * q + 2], outw[4 * q + 3]);
     }
-    for (int j = 0; j < d.k; ++j) {
-      const int pos = j < 32 ? __shfl_sync(0xffffffffu, my_pos, j) : w.pair_pos[(size_t)t * d.k + j];
-      __half* xo = w.x16 + (size_t)pos * d.H;
 #pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const int g = g0 + u * 32;
-        if (g < ng) {
+    for (int u = 0; u < kB; ++u) {
+      const int g = g0 + u * 32;
+      if (g < ng) {
 #pragma unroll
-          for (int q = 0; q < G / 8; ++q) reinterpret_cast<uint4*>(xo + g * G)[q] = out[u][q];
-        }
+        for (int q = 0; q < G / 8; ++q) stage[(g - gb) * (G / 8) + q] = out[u][q];
       }
     }
+    // the generic-proxy stores above become visible to the bulk copies
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    const uint32_t bytes = (uint32_t)(min(ng - gb, kB * 32) * G * 2);   // multiple of 64
+    for (int j = 0; j < d.k; ++j) {
+      const int pos = j < 32 ? __shfl_sync(0xffffffffu, my_pos, j) : w.pair_pos[(size_t)t * d.k + j];
+      if (lane == 0) {
+        __half* dst = w.x16 + (size_t)pos * d.H + (size_t)gb * G;     // 64-byte aligned
+        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                     "r"((uint32_t)__cvta_generic_to_shared(stage)), "r"(bytes)
+                     : "memory");
+      }
+    }
+    if (lane == 0) {
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // the buffer may be reused
+    }
+    __syncwarp();
   }
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Step 5: y[t, c] = sum_j p_{t,j} o_{t*k+j}[c], added in selection order j.
