@@ -61,7 +61,7 @@ __device__ __forceinline__ void route_token(const float* __restrict__ row, int E
   float mv;
   int mi;
   rescan(mv, mi);
-  float l0 = 0.f, sum = 0.f;
+  float l0 = 0.f, sum = 0.f, my_z = 0.f;
   for (int j = 0; j < k; ++j) {
     // warp-wide best of the lanes' bests: the largest key, then among the
     // lanes holding it the lowest expert index (two warp reductions)
@@ -78,13 +78,15 @@ __device__ __forceinline__ void route_token(const float* __restrict__ row, int E
     sum += z;                                   // same value in every lane
     if ((j & 31) == lane) {
       idx[j] = bi;
-      pw[j] = z;
+      if (j < 32) my_z = z;
+      else pw[j] = z;
     }
     if (lane == 0) on_pick(bi);
   }
   const float inv = 1.0f / sum;
+  if (lane < k) pw[lane] = my_z * inv;        // p_j = z_j / sum, written once
   __syncwarp();
-  for (int j = lane; j < k; j += 32) pw[j] *= inv;
+  for (int j = 32 + lane; j < k; j += 32) pw[j] *= inv;
 }
 
 template <int PER>
@@ -372,18 +374,19 @@ combine_kernel(Dims d, const float* __restrict__ pw, const __half* __restrict__ 
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   const size_t base = (size_t)t * d.k;
-  for (int j0 = 0; j0 < d.k; j0 += 4) {
-    uint4 raw[4];
-    float p[4];
+  constexpr int kJ = 4;                       // rows whose loads are issued before the first FMA
+  for (int j0 = 0; j0 < d.k; j0 += kJ) {
+    uint4 raw[kJ];
+    float p[kJ];
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
+    for (int jj = 0; jj < kJ; ++jj) {
       if (j0 + jj < d.k) {
         raw[jj] = __ldg(reinterpret_cast<const uint4*>(o16 + (base + j0 + jj) * d.H + c));
         p[jj] = __ldg(pw + base + j0 + jj);
       }
     }
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
+    for (int jj = 0; jj < kJ; ++jj) {
       if (j0 + jj < d.k) {
         const uint32_t wv[4] = {raw[jj].x, raw[jj].y, raw[jj].z, raw[jj].w};
 #pragma unroll
