@@ -162,17 +162,28 @@ def dist_setup(args):
     return world, rank, local
 
 
+def oracle_host():
+    """The oracle's thread count (it is single-threaded) and this host."""
+    from oracle import moe_oracle as O
+    model = "unknown CPU"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return 1, f"{model}, {O.hardware_concurrency()} hardware threads"
+
+
 def bench_reference(args, wl, world, rank):
-    """The float64 oracle as it stands, on the host cores (rank 0 only)."""
+    """The float64 C++ oracle as it stands, single-threaded on a host core
+    (rank 0 only); each step's time is the oracle's own std::chrono figure."""
     if rank != 0:
         return
     from oracle import moe_oracle as O
-    try:
-        import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        cores = max([i.get("num_threads", 1) for i in info] or [1])
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count() or 1
+    cores, host = oracle_host()
     inp = synth.make_inputs(wl)
     nb = synth.expert_bytes(wl.fmt, wl.H, wl.I)
     blobs = [inp.blobs[e, :nb] for e in range(wl.E)]
@@ -181,17 +192,15 @@ def bench_reference(args, wl, world, rank):
 
     def step():
         toks = rng.integers(0, wl.T, ntok)
-        O.moe_prefill_tokens(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I, wl.k, toks)
+        return O.moe_prefill_tokens_timed(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I, wl.k, toks)[3]
 
     for _ in range(args.warmup):
         step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = time.perf_counter() - t0
+    dt = sum(step() for _ in range(args.steps))
     value = args.steps * ntok * wl.k / dt
     sample = (f"{ntok} tokens x top-{wl.k} of the {wl.name} workload per step (routing, decode of "
-              f"the selected experts, float64 FFN, ordered combine), {args.steps} steps")
+              f"the selected experts, float64 FFN, ordered combine), {args.steps} steps; "
+              f"single-threaded C++ oracle on {host}")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -205,27 +214,23 @@ def bench_reference(args, wl, world, rank):
 
 
 def cpu_baseline(wl, budget_s=15.0):
-    """The oracle on a bounded sample of the workload, single process."""
+    """The C++ oracle on a bounded sample of the workload, single-threaded;
+    the time is the sum of the oracle's own std::chrono figures."""
     from oracle import moe_oracle as O
-    try:
-        import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        cores = max([i.get("num_threads", 1) for i in info] or [1])
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count() or 1
+    cores, host = oracle_host()
     inp = synth.make_inputs(wl)
     nb = synth.expert_bytes(wl.fmt, wl.H, wl.I)
     blobs = [inp.blobs[e, :nb] for e in range(wl.E)]
     rng = np.random.default_rng(1)
     done = 0
-    t0 = time.perf_counter()
-    while time.perf_counter() - t0 < budget_s:
+    dt = 0.0
+    while dt < budget_s:
         toks = rng.integers(0, wl.T, 2)
-        O.moe_prefill_tokens(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I, wl.k, toks)
+        dt += O.moe_prefill_tokens_timed(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I, wl.k, toks)[3]
         done += 2
-    dt = time.perf_counter() - t0
     return {"value": done * wl.k / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{done} tokens ({done * wl.k} pairs) of {wl.name}, {dt:.1f} s, float64"}
+            "sample": f"{done} tokens ({done * wl.k} pairs) of {wl.name}, {dt:.1f} s, float64, "
+                      f"single-threaded C++ oracle on {host}"}
 
 
 def bench_ours(args, wl, world, rank, local):
