@@ -373,7 +373,8 @@ def bench_ours(args, wl, world, rank, local):
     value = replica_throughput(world, args.steps, P, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": ms_step, "ms_per_step_median": statistics.median(step_ms),
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
                    "format": synth.FMT_NAMES[wl.fmt], "pairs": P, "touched_experts": touched,
