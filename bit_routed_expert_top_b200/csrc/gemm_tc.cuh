@@ -770,46 +770,5 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
   }
 }
 
-inline int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
-template <int FMT, bool GATEUP>
-int launch(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& bmap, cudaStream_t s,
-           bool pdl) {
-  static bool configured = false;
-  constexpr int smem = smem_bytes<FMT>();
-  if (!configured) {
-    const cudaError_t e = cudaFuncSetAttribute(decode_gemm_kernel<FMT, GATEUP>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return RL_ERR_CUDA;
-    configured = true;
-  }
-  const int maxu = GATEUP ? d.max_units_gu : d.max_units_dn;
-  const int grid = maxu < num_sms() ? maxu : num_sms();
-  return launch_k(decode_gemm_kernel<FMT, GATEUP>, dim3(grid), dim3(kThreads), smem, s, pdl, d, w, tab, bmap) ==
-                 cudaSuccess
-             ? RL_OK
-             : RL_ERR_CUDA;
-}
-
-template <int FMT>
-int launch_gateup(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& xmap, cudaStream_t s,
-                  bool pdl) {
-  return launch<FMT, true>(d, w, tab, xmap, s, pdl);
-}
-template <int FMT>
-int launch_down(const Dims& d, const Work& w, const ExpertTable& tab, const CUtensorMap& hmap, cudaStream_t s,
-                bool pdl) {
-  return launch<FMT, false>(d, w, tab, hmap, s, pdl);
-}
-
 }  // namespace tc
 }  // namespace rl

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -33,6 +34,49 @@ int cuda_fail(cudaError_t e, const char* what) {
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kMaxDevices = 64;  // devices with cached per-device state
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+
+// SM count of device `dev` (the decode-GEMM grid is one persistent CTA per SM).
+int num_sms(int dev) {
+  static std::atomic<int> cached[kMaxDevices];
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  int n = slot ? cached[dev].load(std::memory_order_relaxed) : 0;
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (slot) cached[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+// One decode-GEMM launch.  The kernel takes more than 48 KB of dynamic
+// shared memory, an attribute that belongs to each device's context: it is
+// set once per device (setting it twice from racing threads is harmless).
+template <int FMT, bool GATEUP>
+int launch_decode_gemm(const rl::Dims& d, const rl::Work& w, const rl::ExpertTable& tab, const CUtensorMap& bmap,
+                       cudaStream_t s, bool pdl) {
+  static std::atomic<unsigned long long> configured{0};
+  constexpr int smem = rl::tc::smem_bytes<FMT>();
+  const int dev = current_device();
+  const unsigned long long bit = dev >= 0 && dev < kMaxDevices ? 1ull << dev : 0ull;
+  if (!(configured.load(std::memory_order_acquire) & bit)) {
+    const cudaError_t e = cudaFuncSetAttribute(rl::tc::decode_gemm_kernel<FMT, GATEUP>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_gemm_kernel)");
+    configured.fetch_or(bit, std::memory_order_release);
+  }
+  const int maxu = GATEUP ? d.max_units_gu : d.max_units_dn;
+  const int sms = num_sms(dev);
+  const cudaError_t e = rl::launch_k(rl::tc::decode_gemm_kernel<FMT, GATEUP>, dim3(maxu < sms ? maxu : sms),
+                                     dim3(rl::tc::kThreads), smem, s, pdl, d, w, tab, bmap);
+  return e == cudaSuccess ? RL_OK : cuda_fail(e, "decode_gemm_kernel launch");
+}
 
 // Work-unit shapes of the decode-GEMM stages (see gemm_tc.cuh).
 constexpr int kNtGateUp = rl::tc::kNtGu;
@@ -205,10 +249,10 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
     if (rc != RL_OK) return rc;
     rc = make_act_map(&hmap, w.h16, d.I, d.P, rl::tc::kNT);
     if (rc != RL_OK) return rc;
-    rc = rl::tc::launch_gateup<FMT>(d, w, tab, xmap, s, pdl);
+    rc = launch_decode_gemm<FMT, true>(d, w, tab, xmap, s, pdl);
     if (rc != RL_OK) return rc;
     mark(3, s);
-    rc = rl::tc::launch_down<FMT>(d, w, tab, hmap, s, pdl);
+    rc = launch_decode_gemm<FMT, false>(d, w, tab, hmap, s, pdl);
     if (rc != RL_OK) return rc;
   }
   mark(4, s);
@@ -241,7 +285,6 @@ int fill_table(const void* const* blobs, int E, rl::ExpertTable* tab) {
 // handle: its device address is looked up with cudaGetSymbolAddress, once per
 // device, with that device current.
 __device__ __align__(256) unsigned char g_noalloc_scratch[RL_NOALLOC_SCRATCH_BYTES];
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
 
