@@ -166,7 +166,11 @@ int rl_moe_check_status(void* workspace, void* stream, unsigned* bits_out);
 /* Stage timing: when enabled, rl_moe_prefill[_ws] records CUDA events on its
  * stream around each kernel; rl_moe_profile_read() synchronizes on the last
  * events and writes up to n stage times in milliseconds (route, group,
- * gate/up, down, combine) plus names via rl_moe_profile_stage_name(). */
+ * gate/up, down, combine) plus names via rl_moe_profile_stage_name().
+ * The switch and the events are process-wide, the events made on the device
+ * current at the first rl_moe_profile_enable(1): a measuring aid for one
+ * thread and one device, not for concurrent callers.  While enabled, the
+ * kernels are launched without overlapping their starts. */
 int rl_moe_profile_enable(int on);
 int rl_moe_profile_read(float* stage_ms, int n);
 const char* rl_moe_profile_stage_name(int i);
