@@ -1,7 +1,7 @@
 """Benchmark of the routed-expert MoE prefill layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--no-cpu-baseline] [--no-graph]
 
 A step is one pass of the whole layer (route, group, gate/up decode-GEMM +
 SwiGLU, down decode-GEMM, combine) over one chunk of synthetic input, through
@@ -11,14 +11,16 @@ is flushed (a 256 MB device write) before every timed step; each step is timed
 with CUDA events on the launching stream.  The metric is routed pairs/s (the
 layer's ms per step is in ms_per_step).  A second timed pass records the
 library's CUDA events between its kernels for the stage times and the gate/up
-kernel's duration (the roofline figure).
+kernel's duration (the roofline figure).  The line also carries the same call
+replayed from a CUDA graph captured once (graph_replay) and the end-to-end
+figure with host copies every step (e2e).
 
 Multi-GPU: the layer does not shard (one GPU per layer call), so --gpus N runs
 N independent replicas, one process per GPU under torchrun; value is the pairs
 of all ranks divided by the slowest rank's time (scaling "weak").
 
---impl reference times the float64 CPU oracle on host cores, each step a
-bounded sample of the same workload (rank 0 only).
+--impl reference times the float64 C++ oracle, single-threaded on a host
+core, each step a bounded sample of the same workload (rank 0 only).
 """
 from __future__ import annotations
 
@@ -354,6 +356,43 @@ def bench_ours(args, wl, world, rank, local):
     t1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+
+    # the same call captured once into a CUDA graph and replayed (the six
+    # launches then cost one graph launch); skipped with --no-graph
+    graph_ms, graph_err = None, None
+    graph = None
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(graph, stream=side):
+                    api.rl_moe_prefill_ws(x, logits, table, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws, side)
+            torch.cuda.synchronize()
+        except Exception as e:  # noqa: BLE001 - reported in the line, every rank agrees below
+            graph, graph_err = None, f"{type(e).__name__}: {e}"[:200]
+        # every rank times the replays only if every rank captured
+        if max_over_ranks(0 if graph is not None else 1, world, dev):
+            graph = None
+            graph_err = graph_err or "capture failed on another rank"
+    if graph is not None:
+        gs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ge = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.warmup):
+            flush.fill_(float(i))
+            graph.replay()
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            gs[i].record(stream)
+            graph.replay()
+            ge[i].record(stream)
+        torch.cuda.synchronize()
+        graph_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(gs, ge)), world, dev)
+        bits = api.rl_moe_check_status(ws, stream)
+        if max_over_ranks(bits, world, dev):
+            raise SystemExit(f"device status 0x{bits:x} on rank {rank}: {api.rl_last_error()}")
+        del graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -402,6 +441,13 @@ def bench_ours(args, wl, world, rank, local):
         "clocks": clocks,
         "wall_s_timed_region": wall,
     }
+    if graph_err is not None:
+        line["graph_replay"] = {"error": graph_err}
+    if graph_ms is not None:
+        line["graph_replay"] = {"value": replica_throughput(world, args.steps, P, graph_ms), "unit": UNIT,
+                                "ms_per_step": graph_ms / args.steps,
+                                "method": "rl_moe_prefill_ws captured once into a CUDA graph, replayed every "
+                                          "step (inputs resident, L2 flushed outside the graph)"}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)
@@ -416,6 +462,8 @@ def main():
     ap.add_argument("--workload", default=synth.WORKLOADS[synth.HEADLINE].name,
                     choices=[w.name for w in synth.WORKLOADS])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip timing the layer call captured once into a CUDA graph and replayed")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -72,3 +72,39 @@ def test_noalloc_rejects_sizes_beyond_the_fixed_scratch():
                                     torch.cuda.current_stream().cuda_stream)
     assert rc == -2
     assert "scratch" in api.rl_last_error()
+
+
+def test_noalloc_captured_in_a_cuda_graph_and_replayed_on_new_inputs():
+    """The serving use of the entry point: one call captured into a CUDA graph
+    (no allocation may happen inside the capture), then replayed after new
+    inputs (x, logits and expert blobs) are written into the same device
+    buffers; each replay's y equals the workspace entry point's on the
+    buffers' contents."""
+    a = synth.make_inputs(synth.WORKLOADS[1])                 # 2-token verify step
+    b = synth.make_inputs(synth.WORKLOADS[1], seed=4242)      # other draws, same shapes
+    wl = a.wl
+    x, logits, blobs = Hh.to_device(a)
+    table = api.expert_table(blobs, wl.E)
+    y = torch.full((wl.T, wl.H), float("nan"), dtype=torch.float32, device="cuda")
+    # the first call on a device looks up the scratch array: before any capture
+    api.rl_moe_prefill_noalloc(x, logits, table, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            api.rl_moe_prefill_noalloc(x, logits, table, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y,
+                                       stream=side)
+    torch.cuda.synchronize()
+    for inp in (a, b, a):
+        xi, li, bi = Hh.to_device(inp)
+        x.copy_(xi)
+        logits.copy_(li)
+        blobs.copy_(bi)
+        y.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        y_ref = _ws_reference(inp, x, logits, blobs)
+        Hh.assert_y_close(y.cpu().numpy(), y_ref, "graph replay")
+    del graph
