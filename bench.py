@@ -358,16 +358,17 @@ def bench_ours(args, wl, world, rank, local):
     e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
 
     # the same call captured once into a CUDA graph and replayed (the six
-    # launches then cost one graph launch); skipped with --no-graph
+    # launches then cost one graph launch); one GPU only (with a process group
+    # up, other threads make CUDA calls), skipped with --no-graph
     graph_ms, graph_err = None, None
     graph = None
-    if not args.no_graph:
+    if not args.no_graph and world == 1:
         try:
             graph = torch.cuda.CUDAGraph()
             side = torch.cuda.Stream(dev)
             side.wait_stream(stream)
             with torch.cuda.stream(side):
-                with torch.cuda.graph(graph, stream=side):
+                with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
                     api.rl_moe_prefill_ws(x, logits, table, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws, side)
             torch.cuda.synchronize()
         except Exception as e:  # noqa: BLE001 - reported in the line, every rank agrees below
