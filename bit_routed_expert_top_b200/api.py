@@ -95,6 +95,28 @@ def _need_cuda(*ts):
             raise ValueError("device buffers must be CUDA tensors")
 
 
+def _check_buf(t, name: str, dtypes, min_numel: int):
+    """A tensor argument: one of `dtypes`, contiguous, at least `min_numel`
+    elements (the C ABI reads it as a raw pointer).  Integer addresses pass."""
+    if t is None or isinstance(t, int):
+        return
+    if dtypes and t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name}: {t.numel()} elements, at least {min_numel} needed")
+
+
+_X_DTYPES = (torch.bfloat16, torch.int16, torch.uint16)   # bf16 values or their bit patterns
+
+
+def _check_layer_bufs(x, router_logits, y, T, H, E):
+    _check_buf(x, "x", _X_DTYPES, T * H)
+    _check_buf(router_logits, "router_logits", (torch.float32,), T * E)
+    _check_buf(y, "y", (torch.float32,), T * H)
+
+
 def expert_table(blobs, E: int | None = None):
     """Host array of expert pointers: from a CUDA uint8 tensor [E, stride]
     (expert e at row e) or a sequence of CUDA tensors / integer addresses."""
@@ -130,6 +152,7 @@ def alloc_workspace(fmt, T, H, I, E, k, device=None) -> torch.Tensor:
 
 
 def rl_moe_prefill(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, stream=None):
+    _check_layer_bufs(x, router_logits, y, T, H, E)
     _need_cuda(x, router_logits, y)
     table = expert_blobs if isinstance(expert_blobs, ctypes.Array) else expert_table(expert_blobs, E)
     _check(load().rl_moe_prefill(_ptr(x), _ptr(router_logits), ctypes.cast(table, ctypes.c_void_p),
@@ -138,6 +161,8 @@ def rl_moe_prefill(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, stream
 
 def rl_moe_prefill_ws(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, workspace,
                       stream=None):
+    _check_layer_bufs(x, router_logits, y, T, H, E)
+    _check_buf(workspace, "workspace", (), 0)
     _need_cuda(x, router_logits, y, workspace)
     table = expert_blobs if isinstance(expert_blobs, ctypes.Array) else expert_table(expert_blobs, E)
     nbytes = workspace.numel() * workspace.element_size()
@@ -149,6 +174,7 @@ def rl_moe_prefill_ws(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, wor
 def rl_moe_prefill_noalloc(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, stream=None):
     """The layer with the library's fixed device scratch instead of a workspace
     (no allocation on any call; see include/rl_moe.h for its limits)."""
+    _check_layer_bufs(x, router_logits, y, T, H, E)
     _need_cuda(x, router_logits, y)
     table = expert_blobs if isinstance(expert_blobs, ctypes.Array) else expert_table(expert_blobs, E)
     _check(load().rl_moe_prefill_noalloc(_ptr(x), _ptr(router_logits), ctypes.cast(table, ctypes.c_void_p),
@@ -157,6 +183,14 @@ def rl_moe_prefill_noalloc(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y
 
 def rl_moe_route(router_logits, T, E, k, topk_idx, topk_w, offsets, pair_list, pair_pos,
                  workspace, stream=None):
+    P = T * k
+    _check_buf(router_logits, "router_logits", (torch.float32,), T * E)
+    _check_buf(topk_idx, "topk_idx", (torch.int32,), P)
+    _check_buf(topk_w, "topk_w", (torch.float32,), P)
+    _check_buf(offsets, "offsets", (torch.int32,), E + 1)
+    _check_buf(pair_list, "pair_list", (torch.int32,), P)
+    _check_buf(pair_pos, "pair_pos", (torch.int32,), P)
+    _check_buf(workspace, "workspace", (), 0)
     _need_cuda(router_logits, topk_idx, topk_w, offsets, pair_list, pair_pos, workspace)
     nbytes = workspace.numel() * workspace.element_size()
     _check(load().rl_moe_route(_ptr(router_logits), T, E, k, _ptr(topk_idx), _ptr(topk_w),

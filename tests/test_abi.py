@@ -91,3 +91,57 @@ def test_missing_library_fails_loudly(tmp_path):
             api.load(str(tmp_path / "nope.so"))
     finally:
         api._lib = saved
+
+
+def _cpu_layer_args(wl, x_dtype=None):
+    import torch
+    x = torch.zeros((wl.T, wl.H), dtype=x_dtype or torch.int16)
+    logits = torch.zeros((wl.T, wl.E), dtype=torch.float32)
+    y = torch.zeros((wl.T, wl.H), dtype=torch.float32)
+    return x, logits, y
+
+
+def test_binding_accepts_the_call_patterns_of_the_tests_and_bench():
+    """The binding's argument checks pass the dtypes and sizes every caller in
+    this repository uses; with CPU tensors the only complaint left is the
+    device check, raised before any library call."""
+    import torch
+    wl = synth.WORKLOADS[0]
+    ptrs = [0x1000] * wl.E
+    for x_dtype in (torch.int16, torch.uint16, torch.bfloat16):
+        x, logits, y = _cpu_layer_args(wl, x_dtype)
+        ws = torch.zeros(64, dtype=torch.uint8)
+        for call in (lambda: api.rl_moe_prefill(x, logits, ptrs, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y),
+                     lambda: api.rl_moe_prefill(x, logits, ptrs, wl.fmt, 0, wl.H, wl.I, wl.E, wl.k, y),
+                     lambda: api.rl_moe_prefill_ws(x, logits, ptrs, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws),
+                     lambda: api.rl_moe_prefill_noalloc(x, logits, ptrs, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y)):
+            with pytest.raises(ValueError, match="CUDA tensors"):
+                call()
+    T, E, k = wl.T, wl.E, wl.k
+    route_bufs = dict(idx=torch.zeros((T, k), dtype=torch.int32), w=torch.zeros((T, k), dtype=torch.float32),
+                      off=torch.zeros(E + 1, dtype=torch.int32), pl=torch.zeros(max(T * k, 1), dtype=torch.int32),
+                      pp=torch.zeros(max(T * k, 1), dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        api.rl_moe_route(torch.zeros((T, E)), T, E, k, *route_bufs.values(), torch.zeros(8, dtype=torch.uint8))
+
+
+@pytest.mark.parametrize("bad,match", [
+    ("x_float", "x: dtype"), ("logits_f64", "router_logits: dtype"), ("y_half", "y: dtype"),
+    ("y_short", "y: .* at least"), ("x_strided", "x must be contiguous"),
+])
+def test_binding_rejects_wrong_buffers_before_the_library(bad, match):
+    import torch
+    wl = synth.WORKLOADS[0]
+    x, logits, y = _cpu_layer_args(wl)
+    if bad == "x_float":
+        x = torch.zeros((wl.T, wl.H), dtype=torch.float32)
+    elif bad == "logits_f64":
+        logits = logits.double()
+    elif bad == "y_half":
+        y = y.half()
+    elif bad == "y_short":
+        y = y[:-1]
+    elif bad == "x_strided":
+        x = torch.zeros((wl.H, wl.T), dtype=torch.int16).t()
+    with pytest.raises(ValueError, match=match):
+        api.rl_moe_prefill(x, logits, [0x1000] * wl.E, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y)
