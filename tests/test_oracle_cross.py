@@ -116,3 +116,22 @@ def test_oracle_shares_nothing_with_the_cuda_path():
     if os.path.exists(api.LIB_PATH):
         with open(api.LIB_PATH, "rb") as f:
             assert b"orc_" not in f.read()
+
+
+def test_concurrent_calls_give_the_sequential_results():
+    """The oracle keeps no state between calls, so tokens partitioned over
+    threads (the all-core CPU baseline) give bit-identical rows."""
+    import concurrent.futures as cf
+
+    wl = synth.Workload("conc", 16, 256, 128, 12, 3, O.FMT_Q1)
+    inp = synth.make_inputs(wl, seed=77)
+    nb = O.expert_bytes(wl.fmt, wl.H, wl.I)
+    blobs = [inp.blobs[e, :nb] for e in range(wl.E)]
+    parts = [np.arange(i, wl.T, 4) for i in range(4)]
+    seq = [O.moe_prefill_tokens(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I, wl.k, t) for t in parts]
+    with cf.ThreadPoolExecutor(4) as ex:
+        par = list(ex.map(lambda t: O.moe_prefill_tokens(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I,
+                                                         wl.k, t), parts))
+    for a, b in zip(seq, par):
+        for u, v in zip(a, b):
+            assert np.array_equal(u, v)
