@@ -249,7 +249,9 @@ def oracle_all_cores(wl, inp, blobs, budget_s=7.5, threads=None):
     import concurrent.futures as cf
 
     from oracle import moe_oracle as O
-    n = threads or os.cpu_count() or 1
+    # the CPUs this process may run on, at most 32 (each call holds ~25 MB
+    # of decoded expert weights)
+    n = threads or max(1, min(len(os.sched_getaffinity(0)), 32))
 
     def work(seed):
         rng = np.random.default_rng(seed)
