@@ -145,3 +145,26 @@ def test_binding_rejects_wrong_buffers_before_the_library(bad, match):
         x = torch.zeros((wl.H, wl.T), dtype=torch.int16).t()
     with pytest.raises(ValueError, match=match):
         api.rl_moe_prefill(x, logits, [0x1000] * wl.E, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y)
+
+
+def test_header_limits_are_the_library_limits():
+    """RL_MAX_EXPERTS, RL_MAX_DIM and RL_MAX_PAIRS as the header states them
+    bound what rl_moe_workspace_bytes accepts."""
+    src = open(HEADER).read()
+    def value(v):
+        a, _, b = v.partition("<<")
+        return int(a) << int(b) if b else int(a)
+    lim = {n: value(v) for n, v in re.findall(r"#define (RL_MAX_\w+) \(?([0-9 <]+)\)?", src)}
+    assert lim == {"RL_MAX_EXPERTS": 1024, "RL_MAX_DIM": 8192, "RL_MAX_PAIRS": 1 << 24}
+    ok = api.rl_moe_workspace_bytes
+    assert ok(2, 8, 256, 128, lim["RL_MAX_EXPERTS"], 2) > 0
+    assert api.load().rl_moe_workspace_bytes(2, 8, 256, 128, lim["RL_MAX_EXPERTS"] + 1, 2) == 0
+    assert ok(2, 8, lim["RL_MAX_DIM"], lim["RL_MAX_DIM"], 16, 2) > 0
+    assert api.load().rl_moe_workspace_bytes(2, 8, lim["RL_MAX_DIM"] + 32, 128, 16, 2) == 0
+    assert ok(2, lim["RL_MAX_PAIRS"] // 2, 32, 32, 16, 2) > 0
+    assert api.load().rl_moe_workspace_bytes(2, lim["RL_MAX_PAIRS"] // 2 + 1, 32, 32, 16, 2) == 0
+
+
+def test_launch_count_is_the_six_kernels():
+    # route, group, pair placement, gate/up, down, combine
+    assert api.rl_moe_launches_per_call() == 6
