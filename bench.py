@@ -12,8 +12,9 @@ with CUDA events on the launching stream.  The metric is routed pairs/s (the
 layer's ms per step is in ms_per_step).  A second timed pass records the
 library's CUDA events between its kernels for the stage times and the gate/up
 kernel's duration (the roofline figure).  The line also carries the same call
-replayed from a CUDA graph captured once (graph_replay) and the end-to-end
-figure with host copies every step (e2e).
+replayed from a CUDA graph captured once (graph_replay), the end-to-end
+figure with host copies every step (e2e), and (one GPU) the other four
+workloads timed the same way (per_workload).
 
 Multi-GPU: the layer does not shard (one GPU per layer call), so --gpus N runs
 N independent replicas, one process per GPU under torchrun; value is the pairs
@@ -270,6 +271,87 @@ def oracle_all_cores(wl, inp, blobs, budget_s=7.5, threads=None):
             "sample": f"{done} tokens on {n} threads, {wall:.1f} s wall"}
 
 
+def touched_experts(api, torch, logits, wl, ws, dev):
+    """Experts with at least one pair (the byte count of the roofline), from
+    the library's own routing export."""
+    P = wl.T * wl.k
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+    w_ = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+    off = torch.empty(wl.E + 1, dtype=torch.int32, device=dev)
+    pl = torch.empty(P, dtype=torch.int32, device=dev)
+    pp = torch.empty(P, dtype=torch.int32, device=dev)
+    api.rl_moe_route(logits, wl.T, wl.E, wl.k, idx, w_, off, pl, pp, ws)
+    return int((torch.diff(off) > 0).sum().item())
+
+
+def per_workload_figures(args, dev, flush, headline):
+    """The other workloads of the layer, each timed like the headline (L2
+    flushed before every step, CUDA events around each call on the launching
+    stream) and replayed from a CUDA graph: median ms per call, routed
+    pairs/s, and the fraction of its own roofline."""
+    import torch
+    from bit_routed_expert_top_b200 import api
+
+    peaks, _ = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for wl in synth.WORKLOADS:
+        if wl.name == headline:
+            continue
+        inp = synth.make_inputs(wl)
+        x = torch.from_numpy(inp.x_bits.view(np.int16).copy()).to(dev)
+        logits = torch.from_numpy(inp.logits).to(dev)
+        blobs = torch.from_numpy(inp.blobs).to(dev)
+        table = api.expert_table(blobs, wl.E)
+        y = torch.empty((wl.T, wl.H), dtype=torch.float32, device=dev)
+        ws = api.alloc_workspace(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, device=dev)
+
+        def call(s=stream):
+            api.rl_moe_prefill_ws(x, logits, table, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws, s)
+
+        def timed(fn):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for i in range(args.warmup):
+                flush.fill_(float(i))
+                fn()
+            for i, (a, b) in enumerate(ev):
+                flush.fill_(float(i))
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            return [a.elapsed_time(b) for a, b in ev]
+
+        ms = timed(call)
+        bits = api.rl_moe_check_status(ws, stream)
+        if bits:
+            raise SystemExit(f"device status 0x{bits:x} on {wl.name}: {api.rl_last_error()}")
+        graph_ms = None
+        if not args.no_graph:
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(g, stream=side, capture_error_mode="thread_local"):
+                    call(side)
+            torch.cuda.synchronize()
+            graph_ms = statistics.median(timed(g.replay))
+            del g
+        touched = touched_experts(api, torch, logits, wl, ws, dev)
+        model = layer_model(wl, touched)
+        t_roof = max(model["flops"] / (peaks["bf16_tflops"] * 1e12), model["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+        med = statistics.median(ms)
+        out[wl.name] = {"T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "format": synth.FMT_NAMES[wl.fmt],
+                        "ms_median": med, "ms_mean": statistics.mean(ms), "pairs_per_s": wl.T * wl.k / (med * 1e-3),
+                        "touched_experts": touched, "t_roof_ms": t_roof, "layer_roofline_frac": t_roof / med,
+                        "graph_replay_ms_median": graph_ms,
+                        "graph_layer_roofline_frac": t_roof / graph_ms if graph_ms else None}
+        del x, logits, blobs, y, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def bench_ours(args, wl, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -303,15 +385,7 @@ def bench_ours(args, wl, world, rank, local):
     if max_over_ranks(bits, world, dev):
         raise SystemExit(f"device status 0x{bits:x} on rank {rank}: {api.rl_last_error()}")
 
-    # touched experts (for the byte count of the roofline)
-    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
-    w_ = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
-    off = torch.empty(wl.E + 1, dtype=torch.int32, device=dev)
-    pl = torch.empty(P, dtype=torch.int32, device=dev)
-    pp = torch.empty(P, dtype=torch.int32, device=dev)
-    api.rl_moe_route(logits, wl.T, wl.E, wl.k, idx, w_, off, pl, pp, ws, stream)
-    counts = torch.diff(off).cpu().numpy()
-    touched = int((counts > 0).sum())
+    touched = touched_experts(api, torch, logits, wl, ws, dev)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -429,6 +503,9 @@ def bench_ours(args, wl, world, rank, local):
         if max_over_ranks(bits, world, dev):
             raise SystemExit(f"device status 0x{bits:x} on rank {rank}: {api.rl_last_error()}")
         del graph
+    per_wl = None
+    if world == 1 and not args.no_per_workload:
+        per_wl = per_workload_figures(args, dev, flush, wl.name)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -484,6 +561,8 @@ def bench_ours(args, wl, world, rank, local):
                                 "ms_per_step": graph_ms / args.steps,
                                 "method": "rl_moe_prefill_ws captured once into a CUDA graph, replayed every "
                                           "step (inputs resident, L2 flushed outside the graph)"}
+    if per_wl is not None:
+        line["per_workload"] = per_wl
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)
@@ -500,6 +579,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip timing the layer call captured once into a CUDA graph and replayed")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the figures of the other workloads (one GPU only)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -40,7 +40,11 @@ SIGNATURES = {
 # stage cross-checks of the tensor-core kernels.
 DEBUG_SIGNATURES = {
     "rl_moe_debug_set_gemm": (_i, [_i]),
+    "rl_moe_debug_set_fault": (_i, [_i, ctypes.c_longlong]),
 }
+RL_DEV_UNIT_OVERFLOW = 0x1
+RL_DEV_WAIT_TIMEOUT = 0x2
+RL_DEV_BAD_GROUPING = 0x4
 
 _lib = None
 
@@ -224,6 +228,15 @@ def rl_moe_launches_per_call() -> int:
 
 def rl_last_error() -> str:
     return load().rl_last_error().decode(errors="replace")
+
+
+def debug_set_fault(withhold_b: bool = False, wait_cycles: int = 0):
+    """Test hook of the bounded device waits (not in the public header):
+    with withhold_b the decode-GEMMs' B-operand warp issues no load, so the
+    MMA warp's first wait runs out after wait_cycles SM clock cycles and the
+    call reports RL_DEV_WAIT_TIMEOUT.  wait_cycles <= 0 restores the default
+    limit (about 2 s)."""
+    _check(load().rl_moe_debug_set_fault(1 if withhold_b else 0, int(wait_cycles)))
 
 
 def debug_set_gemm(which: str):

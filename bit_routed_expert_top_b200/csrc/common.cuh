@@ -89,7 +89,17 @@ struct Dims {
   int nt_gu;      // max pairs per gate/up work unit
   int nt_dn;      // max pairs per down work unit
   int max_units_gu, max_units_dn;
+  long long wait_cycles;  // limit of every bounded device wait, in SM clock cycles
+  int debug_fault;        // RL_DEBUG_* bits (0 on every normal call)
 };
+
+// Debug switches of the decode-GEMMs (set by rl_moe_debug_set_fault, never on
+// a normal call): the B-operand warp issues no load at all, so the MMA warp's
+// first wait cannot be satisfied and must run out; the test of the timeout
+// path uses it with a short wait limit.
+constexpr int RL_DEBUG_WITHHOLD_B = 0x1;
+// Default wait limit: about 2 s at the B200's 1.965 GHz boost clock.
+constexpr long long kDefaultWaitCycles = 4000000000LL;
 
 // Device pieces carved from the workspace (or caller buffers for rl_moe_route).
 struct Work {

@@ -88,7 +88,6 @@ constexpr int kDecWarps = 4 * kMT * kDecPhases;  // lane quarters x tiles x phas
 constexpr int kFetchWarp0 = kDecWarp0 + kDecWarps;
 constexpr int kWarps = kFetchWarp0 + kMT;
 constexpr int kThreads = kWarps * 32;
-constexpr long long kWaitCycles = 4000000000LL; // ~2 s at 2 GHz
 constexpr int kUnitCache = 64;                  // this CTA's first work units, cached in shared memory
 constexpr int kSharedBytes = 4096;              // barriers, work-unit cache, pair tokens
 static_assert(kRingCol + kRing * kMT * kSlotCols <= 512, "TMEM columns");
@@ -275,6 +274,7 @@ struct Shared {
   uint64_t acc_full[kAccBufs], acc_empty[kAccBufs], drain;
   uint32_t tmem_base;
   int abort_flag;
+  long long wait_limit;                  // Dims::wait_cycles
   int4 unit[kUnitCache];                 // units blockIdx.x + i*gridDim.x
   const uint8_t* blob[kUnitCache];       // their expert blobs
 };
@@ -295,7 +295,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared*
       const long long now = clock64();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > kWaitCycles) {
+      } else if (now - t0 > sh->wait_limit) {
         *(volatile int*)&sh->abort_flag = 1;
         atomicOr(status, RL_DEV_WAIT_TIMEOUT);
         return false;
@@ -308,6 +308,20 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, Sh
                                               bool sleepy = false) {
   if (__all_sync(0xffffffffu, mbar_try_wait(smem_addr(bar), parity))) return true;
   return __all_sync(0xffffffffu, wait_bar(bar, parity, sh, status, sleepy));
+}
+// Bounded wait that does not give up on the abort flag: used where this
+// thread's own asynchronous operations must have finished before the CTA may
+// leave (MMAs reading TMEM, TMA writes into shared memory).
+__device__ __forceinline__ bool wait_bar_own(uint64_t* bar, uint32_t parity, Shared* sh, unsigned* status) {
+  const uint32_t addr = smem_addr(bar);
+  const long long t0 = clock64();
+  while (!mbar_try_wait(addr, parity)) {
+    if (clock64() - t0 > sh->wait_limit) {
+      atomicOr(status, RL_DEV_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
 }
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
@@ -481,6 +495,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     }
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
+    sh->wait_limit = d.wait_cycles;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -543,14 +558,15 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       if (ok) mma_commit(&sh->acc_full[buf]);
     }
     // drain: every MMA issued by this warp has completed before teardown
+    // (also after an abort: TMEM is freed only once they have run)
     mma_commit(&sh->drain);
-    wait_bar_warp(&sh->drain, 0, sh, w.status);
+    __all_sync(0xffffffffu, wait_bar_own(&sh->drain, 0, sh, w.status));
   } else if (warp == 1) {
     // ------------------------------------------- B operand by TMA --------
     // Lane 0 posts the byte count; lanes 0 and 1 each load one 64-column K
     // block of the unit's kNT activation rows (rows past the end read zeros).
     uint32_t b_it = 0;
-    bool ok = true;
+    bool ok = (d.debug_fault & RL_DEBUG_WITHHOLD_B) == 0;
     for (int ui = 0; ui < my_units && ok; ++ui) {
       const int n0 = unit_at(ui).z;
       for (int kc = 0; kc < nbchunk && ok; ++kc, ++b_it) {
@@ -564,6 +580,13 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
           tma_load_2d(stage + lane * kBBlockBytes, &bmap, kc * kBK + lane * kBKBlock, n0, &sh->full_b[s]);
         __syncwarp();
       }
+    }
+    // after an abort, the loads this warp issued must land before the CTA
+    // leaves: wait for the last load of every stage (a landed stage's phase
+    // has completed whether or not the MMA warp consumed it)
+    if (!ok) {
+      for (uint32_t i = b_it > (uint32_t)kBStages ? b_it - kBStages : 0u; i < b_it; ++i)
+        __all_sync(0xffffffffu, wait_bar_own(&sh->full_b[i % kBStages], (i / kBStages) & 1, sh, w.status));
     }
   } else if (warp < kDecWarp0) {
     // ------------------------------------------------------ epilogue -----
@@ -759,6 +782,8 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
         cp_async_mbar_arrive(&sh->full_raw[s]);
       }
     }
+    // copies still in flight after an abort land before the CTA leaves
+    asm volatile("cp.async.wait_all;" ::: "memory");
   }
 
   tc_fence_before();

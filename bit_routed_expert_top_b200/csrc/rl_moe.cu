@@ -86,6 +86,13 @@ static_assert(kNtGateUp == kNtDown, "the grouping kernel derives both unit lists
 // route, group, pair placement + x gather, gate/up, down, combine
 constexpr int kLaunchesPerCall = 6;
 
+// Debug switches (not in the public header): which decode-GEMM runs (0:
+// tensor cores, 1: CUDA cores), the limit of every bounded device wait, and
+// the RL_DEBUG_* fault bits.  Read once per call into its Dims.
+std::atomic<int> g_gemm{0};
+std::atomic<long long> g_wait_cycles{rl::kDefaultWaitCycles};
+std::atomic<int> g_fault{0};
+
 struct Layout {
   size_t status, idx, pw, bitmap, wprefix, offsets, pair_list, pair_pos, counters, look,
       units_gu, units_dn, x16, h16, o16, total;
@@ -122,6 +129,8 @@ int plan(int fmt, int T, int H, int I, int E, int k, rl::Dims* d, Layout* L) {
   d->nt_dn = kNtDown;
   d->max_units_gu = d->slabs_gu * (E + (d->P + kNtGateUp - 1) / kNtGateUp);
   d->max_units_dn = d->groups_dn * (E + (d->P + kNtDown - 1) / kNtDown);
+  d->wait_cycles = g_wait_cycles.load(std::memory_order_relaxed);
+  d->debug_fault = g_fault.load(std::memory_order_relaxed);
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t at = o; o = align_up(o + bytes, 256); return at; };
   L->status = take(256);
@@ -165,19 +174,20 @@ rl::Work carve(void* ws, const Layout& L) {
 }
 
 // ---- stage timing ----------------------------------------------------------
+// A measuring aid for one thread (see include/rl_moe.h): the switch is
+// atomic so that other threads see a consistent value, the events belong to
+// the thread that enabled it.
 constexpr int kStages = 5;
 const char* kStageNames[kStages] = {"route", "group", "gateup", "down", "combine"};
-bool g_prof = false;
+std::atomic<bool> g_prof{false};
 cudaEvent_t g_ev[kStages + 1];
 bool g_ev_made = false;
-bool g_ev_recorded = false;
+std::atomic<bool> g_ev_recorded{false};
 
 inline void mark(int i, cudaStream_t s) {
-  if (g_prof) cudaEventRecord(g_ev[i], s);
+  if (g_prof.load(std::memory_order_relaxed)) cudaEventRecord(g_ev[i], s);
 }
 
-// Which decode-GEMM implementation runs (0: tensor cores, 1: CUDA cores).
-int g_gemm = 0;
 
 // ---- TMA descriptors of the B operands (x16 for gate/up, h16 for down) -----
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -229,17 +239,18 @@ void launch_route(const float* logits, const rl::Dims& d, const rl::Work& w, cud
 template <int FMT>
 int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
                const rl::Work& w, float* y, cudaStream_t s) {
+  const bool prof = g_prof.load(std::memory_order_relaxed);
   mark(0, s);
   // kernels after the first start while their predecessor drains
   // (programmatic dependent launch), except when stage events sit between
-  const bool pdl = !g_prof;
+  const bool pdl = !prof;
   launch_route(logits, d, w, s);
   mark(1, s);
   rl::launch_k(rl::group_kernel, dim3((d.E + 7) / 8), dim3(256), 0, s, pdl, d, w, 1);
   rl::launch_k(rl::place_pairs_kernel<FMT>, dim3((d.T + 7) / 8), dim3(256), 0, s, pdl,
                static_cast<const uint16_t*>(x), d, w);
   mark(2, s);
-  if (g_gemm == 1) {
+  if (g_gemm.load(std::memory_order_relaxed) == 1) {
     rl::gateup_simt_kernel<FMT><<<d.max_units_gu, 256, 0, s>>>(d, w, tab);
     mark(3, s);
     rl::down_simt_kernel<FMT><<<d.max_units_dn, 256, 0, s>>>(d, w, tab);
@@ -259,7 +270,7 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
   rl::launch_k(rl::combine_kernel, dim3(d.T, (d.H + 1023) / 1024), dim3(128), 0, s, pdl,
                d, static_cast<const float*>(w.pw), static_cast<const __half*>(w.o16), y);
   mark(5, s);
-  if (g_prof) g_ev_recorded = true;
+  if (prof) g_ev_recorded = true;
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return RL_OK;
@@ -466,6 +477,17 @@ int rl_moe_launches_per_call(void) { return kLaunchesPerCall; }
 int rl_moe_debug_set_gemm(int which) {
   if (which != 0 && which != 1) return fail(RL_ERR_INVALID_ARG, "gemm %d", which);
   g_gemm = which;
+  return RL_OK;
+}
+
+// Fault injection for the test of the bounded waits (on the host side of the
+// kernels: a producer that never delivers, never a GPU fault): `fault` is a
+// set of RL_DEBUG_* bits, `wait_cycles` the limit of every device wait
+// (<= 0 restores the default of about 2 s).
+int rl_moe_debug_set_fault(int fault, long long wait_cycles) {
+  if (fault & ~rl::RL_DEBUG_WITHHOLD_B) return fail(RL_ERR_INVALID_ARG, "fault bits 0x%x", fault);
+  g_fault = fault;
+  g_wait_cycles = wait_cycles > 0 ? wait_cycles : rl::kDefaultWaitCycles;
   return RL_OK;
 }
 

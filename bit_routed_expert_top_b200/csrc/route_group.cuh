@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(256) group_kernel(Dims d, Work w, int make_uni
           if ((v >> 62) != 0u) break;
           const long long now = clock64();
           if (t0 == 0) t0 = now;
-          else if (now - t0 > 2000000000LL) {      // ~1 s: give up, flag it
+          else if (now - t0 > d.wait_cycles) {     // give up, flag it
             set_status(w.status, RL_DEV_WAIT_TIMEOUT);
             break;
           }

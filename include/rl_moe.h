@@ -97,8 +97,18 @@ size_t rl_moe_workspace_bytes(int fmt, int T, int H, int I, int E, int k);
  *                 The table is copied by value into the launches, so the
  *                 caller may change or free the host array once the call
  *                 returns (the blobs themselves must live until the stream
- *                 has run the call).
- *   y             device, fp32 [T, H] row-major, overwritten.
+ *                 has run the call).  "Red Lite dev72 - bounded verify,
+ *                 profiling", section 1: the first 2-row verify gave one row
+ *                 the other row's expert tables because the pool kept them in
+ *                 shared buffers that the next encode rewrote; the fix there,
+ *                 as here, hands each call its own copy of the table.
+ *   y             device, fp32 [T, H] row-major, overwritten.  Each token's
+ *                 k expert outputs are added in that token's selection order
+ *                 (dev72 section 1: each row's plan in its own selection
+ *                 order; "Red Lite dev75 - --kv f16, faster prompt
+ *                 ingestion", section 3: the MoE tail sums in selection
+ *                 order).  Routing is exact, with no dependence on cache or
+ *                 other state (dev72 section 1: exact routing only).
  * Draws its workspace from the stream-ordered allocator (cudaMallocAsync on
  * `stream`) and frees it stream-ordered; device status is then not readable,
  * use rl_moe_prefill_ws for that.  T = 0 is a no-op.
@@ -108,8 +118,13 @@ int rl_moe_prefill(const void* x, const float* router_logits,
                    int E, int k, float* y, void* stream);
 
 /* Same, with a caller-owned device workspace of at least
- * rl_moe_workspace_bytes() bytes, 256-byte aligned.  Calls that share a
- * workspace must be ordered on one stream. */
+ * rl_moe_workspace_bytes() bytes, 256-byte aligned (same table-by-value,
+ * selection-order and exact-routing contract as rl_moe_prefill: dev72
+ * section 1, dev75 section 3).  Calls that share a workspace must be ordered
+ * on one stream.  Each call clears the workspace's status word when its
+ * first kernel starts, so rl_moe_check_status reports the problems of the
+ * latest call on that workspace: check after every call whose status
+ * matters. */
 int rl_moe_prefill_ws(const void* x, const float* router_logits,
                       const void* const* expert_blobs, int fmt, int T, int H,
                       int I, int E, int k, float* y, void* workspace,
@@ -147,7 +162,11 @@ int rl_moe_prefill_noalloc(const void* x, const float* router_logits,
                            int E, int k, float* y, void* stream);
 
 /*
- * Steps 1-2 alone (parity/debug export).  Outputs, all device memory:
+ * Steps 1-2 alone (parity/debug export): exact top-k in selection order and
+ * grouping by expert ("Red Lite dev72 - bounded verify, profiling", section
+ * 1: router selection per row, exact routing only; section 3: near-ties
+ * between experts flip the routing, hence exact fp32 comparison with ties to
+ * the lower index).  Outputs, all device memory:
  *   topk_idx int32 [T, k], topk_w fp32 [T, k]  (selection order)
  *   offsets  int32 [E + 1]                     (exclusive prefix of counts)
  *   pair_list int32 [T*k]: pair ids grouped by expert, ascending token
@@ -159,8 +178,9 @@ int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx,
                  void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronizes `stream`, reads and clears the device status word of
- * `workspace`; returns RL_OK, or RL_ERR_DEVICE_STATUS with the bits in
- * *bits_out (may be NULL) and the message in rl_last_error(). */
+ * `workspace`: the RL_DEV_* bits of the latest call on it (each call clears
+ * the word when it starts).  Returns RL_OK, or RL_ERR_DEVICE_STATUS with the
+ * bits in *bits_out (may be NULL) and the message in rl_last_error(). */
 int rl_moe_check_status(void* workspace, void* stream, unsigned* bits_out);
 
 /* Stage timing: when enabled, rl_moe_prefill[_ws] records CUDA events on its

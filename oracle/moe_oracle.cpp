@@ -278,6 +278,34 @@ int orc_moe_prefill(int fmt, const uint16_t* x_bits, const float* logits, const 
   return orc_combine(p, o_all.data(), T, k, H, y);
 }
 
+// Per-pair expert outputs o (pair-id order, [T*k, H]) of the pairs that
+// belong to experts e0 <= e < e1, from the grouped lists of orc_group; rows
+// of other experts' pairs are not written.  Each expert is decoded once and
+// every pair goes through the same ffn_row as in orc_moe_prefill, so calls
+// over disjoint expert ranges (which write disjoint rows, and may run on
+// separate threads) together give orc_moe_prefill's o bit for bit.
+int orc_expert_outputs(int fmt, const uint16_t* x_bits, const uint8_t* const* blobs, int T, int H, int I, int E,
+                       int k, const int32_t* offsets, const int32_t* pair_list, int e0, int e1, double* o) {
+  if (!dims_ok(fmt, H, I) || T < 0 || E < 1 || k < 1 || !blobs || !offsets || e0 < 0 || e1 > E || e0 > e1)
+    return -1;
+  if (T && (!x_bits || !pair_list || !o)) return -1;
+  std::vector<double> x((size_t)H), hrow((size_t)I);
+  Expert ex;
+  for (int e = e0; e < e1; ++e) {
+    if (offsets[e] == offsets[e + 1]) continue;
+    if (!blobs[e]) return -1;
+    decode_expert(fmt, blobs[e], H, I, &ex);
+    for (int64_t pos = offsets[e]; pos < offsets[e + 1]; ++pos) {
+      const int64_t q = pair_list[pos];
+      const int64_t t = q / k;
+      if (t < 0 || t >= T) return -1;
+      for (int c = 0; c < H; ++c) x[c] = bf16_to_double(x_bits[t * H + c]);
+      ffn_row(ex.wg.data(), ex.wu.data(), ex.wd.data(), H, I, x.data(), hrow.data(), o + q * H);
+    }
+  }
+  return 0;
+}
+
 // y rows of n tokens given by their own rows (a token's output depends only
 // on its x row and logit row): x_rows bf16 [n,H], logit_rows fp32 [n,E] ->
 // idx [n,k], p [n,k], y [n,H].  Each pair decodes its expert anew.  When

@@ -62,6 +62,7 @@ _SIGNATURES = {
     "orc_combine": (_i, [_p, _p, _i, _i, _i, _p]),
     "orc_moe_prefill": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p]),
     "orc_moe_prefill_tokens": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
+    "orc_expert_outputs": (_i, [_i, _p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _i, _p]),
     "orc_hardware_concurrency": (ctypes.c_uint, []),
 }
 
@@ -286,6 +287,42 @@ def moe_prefill_tokens(x_bits, logits, blobs, fmt: int, H: int, I: int, k: int, 
     """Returns (idx [n, k], p [n, k], y [n, H]) of the given tokens."""
     idx, p, y, _ = moe_prefill_tokens_timed(x_bits, logits, blobs, fmt, H, I, k, tokens)
     return idx, p, y
+
+
+def moe_prefill_threaded(x_bits, logits, blobs, fmt: int, H: int, I: int, k: int, threads: int = 0):
+    """The whole layer with the per-pair expert outputs computed over host
+    threads, each thread a range of experts (orc_expert_outputs); routing,
+    grouping and the ordered combine are the single-threaded oracle calls.
+    The result equals moe_prefill's bit for bit (every pair's arithmetic is
+    the same); only the work is spread.  Returns idx, p, offsets, pair_list,
+    pair_pos and y."""
+    import concurrent.futures as cf
+
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    if x_bits.shape != (T, H) or len(blobs) != E or not 1 <= k <= E:
+        raise ValueError("inconsistent shapes")
+    idx, p = route(logits, k)
+    offsets, pair_list, pair_pos = group(idx, E)
+    o = np.zeros((T * k, H), np.float64)
+    _keep, table = _blob_table(blobs)
+    n = threads or max(1, min(len(os.sched_getaffinity(0)), 32))
+    # expert ranges of about equal pair counts (plus one decode per expert)
+    cost = np.diff(offsets).astype(np.float64) + 8.0 * (np.diff(offsets) > 0)
+    cuts = np.searchsorted(np.cumsum(cost), np.linspace(0, cost.sum(), n + 1)[1:-1])
+    bounds = [0, *[int(c) + 1 for c in cuts], E]
+    ranges = [(a, b) for a, b in zip(bounds[:-1], bounds[1:]) if b > a]
+
+    def work(r):
+        return load().orc_expert_outputs(fmt, _ptr(x_bits), ctypes.cast(table, ctypes.c_void_p), T, H, I, E, k,
+                                         _ptr(offsets), _ptr(pair_list), r[0], r[1], _ptr(o))
+
+    with cf.ThreadPoolExecutor(len(ranges)) as ex:
+        rcs = list(ex.map(work, ranges))
+    _check(max(abs(rc) for rc in rcs), "expert_outputs")
+    return dict(idx=idx, p=p, offsets=offsets, pair_list=pair_list, pair_pos=pair_pos,
+                y=combine(p, o, k))
 
 
 def hardware_concurrency() -> int:

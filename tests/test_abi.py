@@ -168,3 +168,12 @@ def test_header_limits_are_the_library_limits():
 def test_launch_count_is_the_six_kernels():
     # route, group, pair placement, gate/up, down, combine
     assert api.rl_moe_launches_per_call() == 6
+
+
+def test_fault_switch_accepts_only_known_bits():
+    """The test hook of the bounded waits (no CUDA call): unknown fault bits
+    are refused, the known one and the reset are accepted."""
+    lib = api.load()
+    assert lib.rl_moe_debug_set_fault(0x10, 0) == -1        # RL_ERR_INVALID_ARG
+    assert lib.rl_moe_debug_set_fault(1, 2_000_000) == 0
+    assert lib.rl_moe_debug_set_fault(0, 0) == 0

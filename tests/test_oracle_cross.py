@@ -135,3 +135,34 @@ def test_concurrent_calls_give_the_sequential_results():
     for a, b in zip(seq, par):
         for u, v in zip(a, b):
             assert np.array_equal(u, v)
+
+
+@pytest.mark.parametrize("threads", [1, 3, 7])
+def test_threaded_layer_gives_the_single_threaded_layer_bit_for_bit(threads):
+    """moe_prefill_threaded (per-pair expert outputs over expert ranges on
+    host threads, the full-size parity tests' oracle) against moe_prefill:
+    same arithmetic per pair, so y, routing and lists are identical."""
+    wl = synth.Workload("thr", 40, 256, 96, 13, 3, O.FMT_Q2)
+    inp = synth.make_inputs(wl, seed=91)
+    inp.logits[:, 4] += 3.0                      # one heavy expert, some empty ones
+    nb = O.expert_bytes(wl.fmt, wl.H, wl.I)
+    blobs = [inp.blobs[e, :nb] for e in range(wl.E)]
+    ref = O.moe_prefill(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I, wl.k, keep_intermediates=False)
+    got = O.moe_prefill_threaded(inp.x_bits, inp.logits, blobs, wl.fmt, wl.H, wl.I, wl.k, threads=threads)
+    for key in ("idx", "p", "offsets", "pair_list", "pair_pos", "y"):
+        assert np.array_equal(got[key], ref[key]), key
+
+
+def test_bf16_widening_every_bit_pattern_against_torch():
+    """The oracle's bf16 -> float64 widening for all 65,536 bit patterns
+    against torch's own bf16 -> float64 conversion (a library routine):
+    equal values, equal signs (so -0.0 stays -0.0), NaN exactly where torch
+    gives NaN."""
+    torch = pytest.importorskip("torch")
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = O.bf16_bits_to_f64(bits)
+    want = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(want[~nan]))

@@ -2,9 +2,10 @@
 
 Routing indices, offsets and the expert lists must match bit for bit; the
 routing weights within 1e-6; y within relative L2 5e-3 and
-max|diff| <= 2e-2 * rms(y_ref).  Small cases compare every output; the full
-workloads (launched exactly as bench.py launches them) compare sampled
-tokens, which the oracle computes one by one.
+max|diff| <= 2e-2 * rms(y_ref).  Every case compares every output: the small
+and ragged shapes against the single-threaded oracle, the full-size chunks
+(launched exactly as bench.py launches them) against the same oracle with its
+per-pair expert outputs spread over the host threads.
 """
 import numpy as np
 import pytest
@@ -159,41 +160,105 @@ def test_layer_zero_down_is_zero():
     assert np.all(y == 0.0)
 
 
-def test_intermediates_h_and_o_tiny():
-    inp = synth.make_inputs(synth.WORKLOADS[0])
-    wl = inp.wl
-    y, ws = run_prefill(inp)
-    ref = full_oracle(inp)
+def workspace_h_o(ws, wl):
+    """h (grouped order, K-permutation undone) and o (pair-id order) of the
+    last call, read from the last two pieces of the workspace."""
     n = api.rl_moe_workspace_bytes(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k)
     P = wl.T * wl.k
     raw = ws.cpu().numpy()
     h_bytes = P * wl.I * 2
     o_bytes = P * wl.H * 2
-    # h and o are the last two pieces of the workspace (256-byte aligned)
     o_off = n - ((o_bytes + 255) // 256 * 256)
     h_off = o_off - ((h_bytes + 255) // 256 * 256)
     h = raw[h_off:h_off + h_bytes].view(np.float16).reshape(P, wl.I).astype(np.float64)
     o = raw[o_off:o_off + o_bytes].view(np.float16).reshape(P, wl.H).astype(np.float64)
-    h = Hh.unpermute_k(h, wl.fmt)
+    return Hh.unpermute_k(h, wl.fmt), o
+
+
+def test_intermediates_h_and_o_tiny():
+    inp = synth.make_inputs(synth.WORKLOADS[0])
+    wl = inp.wl
+    y, ws = run_prefill(inp)
+    ref = full_oracle(inp)
+    h, o = workspace_h_o(ws, wl)
     rel_h = np.linalg.norm(h - ref["h"]) / np.linalg.norm(ref["h"])
     rel_o = np.linalg.norm(o - ref["o"]) / np.linalg.norm(ref["o"])
     assert rel_h < 2e-3, rel_h
     assert rel_o < 2e-3, rel_o
 
 
-@pytest.mark.parametrize("wi", [1, 2, 3, 4])
-def test_full_workload_sampled_tokens(wi):
-    """Full-size workloads in bench.py's launch configuration; y of a sample
-    of tokens against the oracle, plus properties at every token."""
+@pytest.mark.parametrize("wi", [2, 3, 4])
+def test_full_workload_every_output(wi):
+    """The three full-size chunks (512 and 2,048 tokens, 512 experts, top-10;
+    Q2 and the skewed Q1), launched as bench.py launches them: every element
+    of y against the oracle (the per-pair outputs computed over the host
+    threads, bit-identical to the single-threaded oracle), plus the routing
+    and the expert lists bit for bit."""
     inp = synth.make_inputs(synth.WORKLOADS[wi])
     wl = inp.wl
-    y, _ = run_prefill(inp)
-    assert np.all(np.isfinite(y))
-    rng = np.random.default_rng(wi)
-    toks = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 10)]))[:12]
-    _, _, yref = O.moe_prefill_tokens(inp.x_bits, inp.logits, Hh.oracle_blobs(inp), wl.fmt, wl.H,
-                                      wl.I, wl.k, toks)
-    Hh.assert_y_close(y[toks], yref, wl.name)
+    y, ws = run_prefill(inp)
+    ref = O.moe_prefill_threaded(inp.x_bits, inp.logits, Hh.oracle_blobs(inp), wl.fmt, wl.H, wl.I, wl.k)
+    Hh.assert_y_close(y, ref["y"], wl.name)
+    idx, w, off, pl, pp = run_route(inp.logits, wl.k)
+    np.testing.assert_array_equal(idx, ref["idx"])
+    np.testing.assert_array_equal(off, ref["offsets"])
+    np.testing.assert_array_equal(pl, ref["pair_list"])
+    np.testing.assert_array_equal(pp, ref["pair_pos"])
+
+
+def edge_inputs(wl, seed):
+    """Inputs whose expert blocks mix the generator's blocks with the edge
+    cases the oracle is pinned on (the hand-built blocks): negative d,
+    subnormal d (both signs), d = +-0, the largest sub-scale s = 7 with the
+    extreme codes u in {0, 3} (Q2) or with every shift flag at +1/8 (Q1), and
+    the hand blocks' sub-scale ramp and code patterns.  d keeps the
+    generator's magnitudes where it is normal, so h and o stay in fp16 range."""
+    inp = synth.make_inputs(wl, seed=seed)
+    rng = np.random.default_rng(seed + 1)
+    bb = synth.BLOCK_BYTES[wl.fmt]
+    nb = synth.expert_bytes(wl.fmt, wl.H, wl.I)
+    blk = inp.blobs[:, :nb].reshape(wl.E, nb // bb, bb)          # a view: edits land in blobs
+    cat = rng.integers(0, 8, blk.shape[:2])
+    d = blk[..., 0].astype(np.uint16) | (blk[..., 1].astype(np.uint16) << 8)
+    d = np.where(cat == 1, d | 0x8000, d)                                     # negative normal d
+    sub = rng.integers(1, 0x400, blk.shape[:2]).astype(np.uint16) | (rng.integers(0, 2, blk.shape[:2]) << 15).astype(np.uint16)
+    d = np.where(cat == 2, sub, d)                                            # subnormal d
+    d = np.where(cat == 3, (rng.integers(0, 2, blk.shape[:2]) << 15).astype(np.uint16), d)   # +-0
+    blk[..., 0] = (d & 0xFF).astype(np.uint8)
+    blk[..., 1] = (d >> 8).astype(np.uint8)
+    top = cat == 4
+    blk[top, 2:5] = 0xFF                                                      # every s = 7
+    if wl.fmt == synth.FMT_Q2:
+        bits = rng.integers(0, 2, (int(top.sum()), 64, 4))
+        codes = (bits * 3) << (2 * np.arange(4))                              # u in {0, 3}
+        blk[top, 5:] = codes.sum(axis=2).astype(np.uint8)
+    else:
+        blk[top, 5] = 0xFF                                                    # delta = +1/8 everywhere
+    ramp = cat == 5                                                           # hand block q2_subscale_ramp /
+    blk[ramp, 2:5] = np.array([0x88, 0xC6, 0xFA], np.uint8)                   # q1_ramp_plus patterns
+    blk[ramp, 5 if wl.fmt == synth.FMT_Q2 else 6:] = 0xE4 if wl.fmt == synth.FMT_Q2 else 0xFF
+    if wl.fmt == synth.FMT_Q1:
+        blk[ramp, 5] = 0xAA
+    return inp
+
+
+@pytest.mark.parametrize("wl", [
+    synth.Workload("edge_q2", 96, 512, 256, 12, 3, synth.FMT_Q2),
+    synth.Workload("edge_q1", 96, 512, 256, 12, 3, synth.FMT_Q1),
+    synth.Workload("edge_q2_ragged", 45, 352, 160, 9, 2, synth.FMT_Q2),
+    synth.Workload("edge_q1_ragged", 45, 352, 160, 9, 2, synth.FMT_Q1),
+], ids=lambda w: w.name)
+def test_edge_blocks_every_output(wl):
+    """The decoder on the blocks of the oracle's pins (negative, subnormal and
+    zero d; s = 7 with u in {0, 3}; Q1 with delta = +1/8): y, and the
+    intermediates h and o, element by element against the oracle."""
+    inp = edge_inputs(wl, seed=sum(wl.name.encode()))
+    y, ws = run_prefill(inp)
+    ref = full_oracle(inp)
+    Hh.assert_y_close(y, ref["y"], wl.name)
+    h, o = workspace_h_o(ws, wl)
+    assert Hh.y_errors(h, ref["h"])[0] < 2e-3
+    assert Hh.y_errors(o, ref["o"])[0] < 2e-3
 
 
 def test_tc_matches_simt_stage_path():
