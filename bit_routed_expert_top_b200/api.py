@@ -35,12 +35,23 @@ SIGNATURES = {
     "rl_moe_profile_stage_name": (ctypes.c_char_p, [_i]),
     "rl_moe_launches_per_call": (_i, []),
     "rl_last_error": (ctypes.c_char_p, []),
+    "rl_moe_cache_create": (_i, [_i, _i, _i, _i, _i, _vp, _i, ctypes.POINTER(_vp)]),
+    "rl_moe_cache_destroy": (_i, [_vp]),
+    "rl_moe_cache_prepare": (_i, [_vp, _vp, _i, _vp]),
+    "rl_moe_cache_table": (_i, [_vp, _vp, _i]),
+    "rl_moe_cache_plan": (_i, [_vp, _vp, _i, _i, _vp]),
+    "rl_moe_cache_shape": (_i, [_vp] + [ctypes.POINTER(_i)] * 4),
+    "rl_moe_cache_slot_of": (_i, [_vp, _i, ctypes.POINTER(_i)]),
+    "rl_moe_cache_stats": (_i, [_vp, ctypes.POINTER(ctypes.c_longlong)]),
+    "rl_moe_verify_bounded": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _sz, _vp, _vp]),
 }
+RL_CACHE_HOST_POOL = 0x1
 # Not in the public header: selects the CUDA-core decode-GEMMs for stage-by-
 # stage cross-checks of the tensor-core kernels.
 DEBUG_SIGNATURES = {
     "rl_moe_debug_set_gemm": (_i, [_i]),
     "rl_moe_debug_set_fault": (_i, [_i, ctypes.c_longlong]),
+    "rl_moe_debug_set_path": (_i, [_i]),
 }
 RL_DEV_UNIT_OVERFLOW = 0x1
 RL_DEV_WAIT_TIMEOUT = 0x2
@@ -202,6 +213,81 @@ def rl_moe_route(router_logits, T, E, k, topk_idx, topk_w, offsets, pair_list, p
                                nbytes, _stream(stream)))
 
 
+class ExpertCache:
+    """rl_moe_cache: up to `slots` of the E expert blobs in one device pool,
+    filled from host copies (host_blobs: a uint8 array [E, >= expert bytes]
+    in host memory, pinned for asynchronous copies, kept alive by this
+    object).  host_pool=True keeps the pool in host memory: the bookkeeping
+    alone, for tests without a GPU."""
+
+    def __init__(self, fmt, H, I, E, slots, host_blobs, host_pool=False):
+        import numpy as np
+        self._blobs = host_blobs
+        if isinstance(host_blobs, torch.Tensor):
+            base, stride = host_blobs.data_ptr(), host_blobs.stride(0) * host_blobs.element_size()
+        else:
+            arr = np.ascontiguousarray(host_blobs)
+            self._blobs = arr
+            base, stride = arr.ctypes.data, arr.strides[0]
+        ptrs = (ctypes.c_void_p * E)(*[base + e * stride for e in range(E)])
+        h = ctypes.c_void_p()
+        _check(load().rl_moe_cache_create(fmt, H, I, E, slots, ctypes.cast(ptrs, ctypes.c_void_p),
+                                          RL_CACHE_HOST_POOL if host_pool else 0, ctypes.byref(h)))
+        self.handle, self.E = h, E
+        self._host_only = host_pool
+
+    def close(self):
+        if self.handle:
+            _check(load().rl_moe_cache_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass
+
+    def prepare(self, experts, stream=None):
+        import numpy as np
+        ex = np.ascontiguousarray(np.asarray(experts, dtype=np.int32).ravel())
+        _check(load().rl_moe_cache_prepare(self.handle, ex.ctypes.data, ex.size,
+                                           None if getattr(self, "_host_only", False) else _stream(stream)))
+
+    def table(self):
+        arr = (ctypes.c_void_p * self.E)()
+        _check(load().rl_moe_cache_table(self.handle, ctypes.cast(arr, ctypes.c_void_p), self.E))
+        return arr
+
+    def plan(self, idx):
+        import numpy as np
+        idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+        T, k = idx.shape
+        out = (ctypes.c_void_p * (T * k))()
+        _check(load().rl_moe_cache_plan(self.handle, idx.ctypes.data, T, k, ctypes.cast(out, ctypes.c_void_p)))
+        return [[out[t * k + j] for j in range(k)] for t in range(T)]
+
+    def slot_of(self, expert) -> int:
+        s = ctypes.c_int(0)
+        _check(load().rl_moe_cache_slot_of(self.handle, expert, ctypes.byref(s)))
+        return s.value
+
+    def stats(self) -> dict:
+        out = (ctypes.c_longlong * 4)()
+        _check(load().rl_moe_cache_stats(self.handle, out))
+        return dict(hits=out[0], misses=out[1], bytes_copied=out[2], evictions=out[3])
+
+
+def rl_moe_verify_bounded(cache, x, router_logits, T, k, y, workspace, stream=None):
+    """One bounded step on an ExpertCache; returns the [T, k] selections."""
+    import numpy as np
+    idx = np.empty((T, k), dtype=np.int32)
+    _need_cuda(x, router_logits, y, workspace)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().rl_moe_verify_bounded(cache.handle, _ptr(x), _ptr(router_logits), T, k, _ptr(y), _ptr(workspace),
+                                        nbytes, idx.ctypes.data, _stream(stream)))
+    return idx
+
+
 def rl_moe_check_status(workspace, stream=None) -> int:
     """Returns the device status bits (0 = fine); raises on a CUDA error."""
     bits = ctypes.c_uint(0)
@@ -237,6 +323,13 @@ def debug_set_fault(withhold_b: bool = False, wait_cycles: int = 0):
     call reports RL_DEV_WAIT_TIMEOUT.  wait_cycles <= 0 restores the default
     limit (about 2 s)."""
     _check(load().rl_moe_debug_set_fault(1 if withhold_b else 0, int(wait_cycles)))
+
+
+def debug_set_path(which: str):
+    """'auto' (chunks of at most 64 pairs take the two-launch decode-regime
+    path where their shapes fit it; the default) or 'prefill' (always the
+    six-launch prefill path)."""
+    _check(load().rl_moe_debug_set_path({"auto": 0, "prefill": 1}[which]))
 
 
 def debug_set_gemm(which: str):

@@ -9,8 +9,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 OUT = os.path.join(PKG, "librl_moe.so")
-SOURCES = ["rl_moe.cu"]
-HEADERS = ["common.cuh", "route_group.cuh", "gemm_simt.cuh", "gemm_tc.cuh"]
+SOURCES = ["rl_moe.cu", "expert_cache.cu"]
+HEADERS = ["common.cuh", "route_group.cuh", "gemm_simt.cuh", "gemm_tc.cuh", "small_t.cuh"]
 
 
 def nvcc():

@@ -117,7 +117,7 @@ struct Work {
   int4* units_dn;        // {expert, slab group, first grouped position, pairs}
   __half* x16;           // [P][H] x of the pair at each grouped position, fp16, K-permuted per group
   __half* h16;           // [P][I] h, grouped order, K-permuted per group
-  __half* o16;           // [P][H] o, pair-id order
+  __half* o16;           // [P][H] o, grouped order
 };
 
 // Programmatic dependent launch: a kernel launched with

@@ -111,7 +111,6 @@ __global__ void __launch_bounds__(256) down_simt_kernel(Dims d, Work w, ExpertTa
   const int4 un = w.units_dn[u];
   const int e = un.x, grp = un.y, n0 = un.z, cnt = un.w;
   __shared__ float hs[32][kSubVals + 1];
-  __shared__ int pids[32];
   const int tid = threadIdx.x;
   const size_t row_bytes = (size_t)d.nbI * d.bb;
   const uint8_t* down = tab.p[e] + (size_t)2 * d.I * d.nbH * d.bb;
@@ -125,7 +124,6 @@ __global__ void __launch_bounds__(256) down_simt_kernel(Dims d, Work w, ExpertTa
     for (int c0 = 0; c0 < cnt; c0 += 32) {
       const int nc = min(32, cnt - c0);
       __syncthreads();
-      if (tid < 32) pids[tid] = tid < nc ? w.pair_list[n0 + c0 + tid] : 0;
       float acc[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc[i] = 0.f;
@@ -152,7 +150,7 @@ __global__ void __launch_bounds__(256) down_simt_kernel(Dims d, Work w, ExpertTa
       }
       if (valid) {
         for (int i = 0; i < nc; ++i)
-          w.o16[(size_t)pids[i] * d.H + r] = __float2half_rn(acc[i]);
+          w.o16[(size_t)(n0 + c0 + i) * d.H + r] = __float2half_rn(acc[i]);   // grouped order
       }
     }
   }

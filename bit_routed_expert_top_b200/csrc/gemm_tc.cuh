@@ -45,6 +45,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace rl {
@@ -335,7 +337,9 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
 template <int FMT>
 __device__ __forceinline__ void make_lut(float dd, uint32_t S, uint32_t flags, int i, uint32_t& lo,
                                          uint32_t& hi) {
-  const float m = dd * (float)(2u * ((S >> (3 * i)) & 7u) + 1u);
+  // s as an exact float from the 2^23 bit pattern, then m = d(2s+1) (exact)
+  const float sf = __uint_as_float(0x4B000000u | ((S >> (3 * i)) & 7u)) - 8388608.0f;
+  const float m = fmaf(sf, 2.0f * dd, dd);
   if constexpr (FMT == RL_FMT_Q2) {
     const __half2 p = __floats2half2_rn(m, 3.0f * m);          // u=2 (low), u=3 (high)
     hi = *reinterpret_cast<const uint32_t*>(&p);
@@ -418,6 +422,55 @@ __device__ __forceinline__ void load16_unaligned(const uint8_t* region, int o, u
   wv[3] = __funnelshift_r(x3, x4, s);
 }
 
+// Code words of one decode step at byte offset o of a row region: Q2 four
+// words (16 bytes), Q1 two (8 bytes).  MODE 0: o is per lane (selects on
+// o & 4); MODE 1 / 2: o & 7 is the same in every lane of the warp and
+// (o & 4) is 0 / 4, so the words are picked without selects.  The shift
+// (o & 3) * 8 is a register in every mode.
+template <int FMT, int MODE>
+__device__ __forceinline__ void load_codes(const uint8_t* region, int o, uint32_t* cw) {
+  if constexpr (MODE == 0) {
+    if constexpr (FMT == RL_FMT_Q2) {
+      uint32_t wv[4];
+      load16_unaligned(region, o, wv);
+      cw[0] = wv[0]; cw[1] = wv[1]; cw[2] = wv[2]; cw[3] = wv[3];
+    } else {
+      load8_unaligned(region, o, cw[0], cw[1]);
+    }
+  } else {
+    const uint8_t* p = region + (o & ~7);
+    const uint32_t s = (uint32_t)(o & 3) * 8u;
+    const uint2 a = *reinterpret_cast<const uint2*>(p);
+    const uint2 b = *reinterpret_cast<const uint2*>(p + 8);
+    if constexpr (FMT == RL_FMT_Q2) {
+      const uint2 c = *reinterpret_cast<const uint2*>(p + 16);
+      if constexpr (MODE == 1) {
+        cw[0] = __funnelshift_r(a.x, a.y, s); cw[1] = __funnelshift_r(a.y, b.x, s);
+        cw[2] = __funnelshift_r(b.x, b.y, s); cw[3] = __funnelshift_r(b.y, c.x, s);
+      } else {
+        cw[0] = __funnelshift_r(a.y, b.x, s); cw[1] = __funnelshift_r(b.x, b.y, s);
+        cw[2] = __funnelshift_r(b.y, c.x, s); cw[3] = __funnelshift_r(c.x, c.y, s);
+      }
+    } else {
+      if constexpr (MODE == 1) {
+        cw[0] = __funnelshift_r(a.x, a.y, s); cw[1] = __funnelshift_r(a.y, b.x, s);
+      } else {
+        cw[0] = __funnelshift_r(a.y, b.x, s); cw[1] = __funnelshift_r(b.x, b.y, s);
+      }
+    }
+  }
+}
+
+// Raw staging: row r of M tile t at tile t's region, even rows first, then
+// odd rows (each half 64 rows x PITCH).  With the odd rows' blocks 8 bytes
+// off the even rows' (rows 552 bytes apart), the 8-byte loads of a
+// half-warp then hit 16 different bank pairs.
+template <int FMT>
+__device__ __forceinline__ int raw_row_offset(int t, int r) {
+  constexpr int PITCH = Raw<FMT>::kPitch;
+  return (t * 128 + (r & 1) * 64 + (r >> 1)) * PITCH;
+}
+
 // Rows of a unit.  GATEUP: unit {expert, slab, n0, cnt}: tile 0 = gate rows
 // 128*slab + r, tile 1 = up rows 128*slab + r, K = H.  DOWN: unit
 // {expert, group, n0, cnt}: tile t = down rows 128*(2*group+t) + r, K = I.
@@ -449,7 +502,6 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
   Shared* sh = reinterpret_cast<Shared*>(b_base + kBStages * kBStageBytes);
 
   constexpr int BB = Fmt<FMT>::kBytes;
-  constexpr int PITCH = Raw<FMT>::kPitch;
   constexpr int CHUNKS = Raw<FMT>::kChunks;
   // the unit count is read from memory: broadcast it from lane 0 so that
   // every loop bound derived from it is provably warp-uniform
@@ -593,18 +645,10 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-    static_assert(kNT <= 64, "the down epilogue keeps two pair ids per lane");
     for (int ui = 0; ui < my_units; ++ui) {
       const int4 un = unit_at(ui);
       const int buf = ui & 1;
       const int cnt = un.w, n0 = un.z;
-      // down: the unit's pair ids (o rows), lane l holding pairs l and 32 + l,
-      // loaded before the wait
-      int pid_lo = 0, pid_hi = 0;
-      if (!GATEUP) {
-        if (lane < cnt) pid_lo = __ldg(w.pair_list + n0 + lane);
-        if (32 + lane < cnt) pid_hi = __ldg(w.pair_list + n0 + 32 + lane);
-      }
       if (!wait_bar_warp(&sh->acc_full[buf], (ui / kAccBufs) & 1, sh, w.status, true)) break;
       tc_fence_after();
       const uint32_t acc0 = tmem + lane_addr + buf * (kMT * kNT);
@@ -628,15 +672,17 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
             }
           }
         } else {
+          // o in grouped order: the unit's pairs are consecutive rows of o16,
+          // so a lane's stores are H apart (the combine finds each pair's row
+          // through pair_pos)
           const int r0 = (un.y * kMT) * 128 + r;
-          const int r1 = r0 + 128;
+          __half* op = w.o16 + (size_t)(n0 + cc * 16) * d.H + r0;
+          const bool ok0 = r0 < d.H, ok1 = r0 + 128 < d.H;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = cc * 16 + j;
-            const int pid = __shfl_sync(0xffffffffu, n < 32 ? pid_lo : pid_hi, n & 31);
-            if (n < cnt) {
-              if (r0 < d.H) w.o16[(size_t)pid * d.H + r0] = __float2half_rn(__uint_as_float(a0[j]));
-              if (r1 < d.H) w.o16[(size_t)pid * d.H + r1] = __float2half_rn(__uint_as_float(a1[j]));
+            if (cc * 16 + j < cnt) {
+              if (ok0) op[(size_t)j * d.H] = __float2half_rn(__uint_as_float(a0[j]));
+              if (ok1) op[(size_t)j * d.H + 128] = __float2half_rn(__uint_as_float(a1[j]));
             }
           }
         }
@@ -653,7 +699,10 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     const int q = warp & 3;                   // TMEM lane quarter
     const int r = q * 32 + lane;              // lane = row inside the tile
     const uint32_t a_col = tmem + ((uint32_t)(q * 32) << 16) + kRingCol + tile * kSlotCols;
-    uint8_t* const my_region0 = raw_base + (tile * 128 + r) * PITCH;
+    uint8_t* const my_region0 = raw_base + raw_row_offset<FMT>(tile, r);
+    // rows a multiple of 8 bytes long: a block's offset mod 8 is the same in
+    // every row (blobs are 16-byte aligned), so the code loads need no selects
+    const bool uniform8 = (rowbytes % 8) == 0;
     const int total_blocks = my_units * nblk;
     bool ok = true;
 
@@ -686,44 +735,53 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       // linear index is its phase mod kDecPhases
       const int m = (int)((ring_it + 4u * kb) % kDecPhases);
       const int j0 = (phase - m + kDecPhases) % kDecPhases;
-      for (int j = j0; j < 4; j += kDecPhases) {
-        const int st = kb * 4 + j;
-        if (2 * st >= nsub) break;
-        const int i = 2 * j;                   // first sub-block of the step inside the block
-        const uint32_t ai = ring_it + st;
-        const int as = ai % kRing;
-        // test the ring slot now; the answer is needed only after the decode
-        const bool slot_free = mbar_test_wait(smem_addr(&sh->empty_a[as]), ((ai / kRing) & 1) ^ 1);
-        // rows past the matrix decode stale stage bytes: their accumulator
-        // rows (TMEM lanes) are never read by the epilogue
-        uint32_t words[32];
-        uint32_t lo0, hi0, lo1, hi1;
-        make_lut<FMT>(dd, S, flags, i, lo0, hi0);
-        make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
-        if constexpr (FMT == RL_FMT_Q2) {
-          uint32_t cw[4];
-          load16_unaligned(region, off + 5 + 8 * i, cw);
-          decode_word<FMT>(cw[0], lo0, hi0, words);
-          decode_word<FMT>(cw[1], lo0, hi0, words + 8);
-          decode_word<FMT>(cw[2], lo1, hi1, words + 16);
-          decode_word<FMT>(cw[3], lo1, hi1, words + 24);
-        } else {
-          uint32_t c0, c1;
-          load8_unaligned(region, off + 6 + 4 * i, c0, c1);
-          decode_word<FMT>(c0, lo0, hi0, words);
-          decode_word<FMT>(c1, lo1, hi1, words + 16);
+      auto steps = [&](auto mode_tag) {
+        constexpr int MODE = decltype(mode_tag)::value;
+        for (int j = j0; j < 4; j += kDecPhases) {
+          const int st = kb * 4 + j;
+          if (2 * st >= nsub) break;
+          const int i = 2 * j;                   // first sub-block of the step inside the block
+          const uint32_t ai = ring_it + st;
+          const int as = ai % kRing;
+          // test the ring slot now; the answer is needed only after the decode
+          const bool slot_free = mbar_test_wait(smem_addr(&sh->empty_a[as]), ((ai / kRing) & 1) ^ 1);
+          // rows past the matrix decode stale stage bytes: their accumulator
+          // rows (TMEM lanes) are never read by the epilogue
+          uint32_t words[32];
+          uint32_t lo0, hi0, lo1, hi1;
+          make_lut<FMT>(dd, S, flags, i, lo0, hi0);
+          make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
+          if constexpr (FMT == RL_FMT_Q2) {
+            uint32_t cw[4];
+            load_codes<FMT, MODE>(region, off + 5 + 8 * i, cw);
+            decode_word<FMT>(cw[0], lo0, hi0, words);
+            decode_word<FMT>(cw[1], lo0, hi0, words + 8);
+            decode_word<FMT>(cw[2], lo1, hi1, words + 16);
+            decode_word<FMT>(cw[3], lo1, hi1, words + 24);
+          } else {
+            uint32_t cw[2];
+            load_codes<FMT, MODE>(region, off + 6 + 4 * i, cw);
+            decode_word<FMT>(cw[0], lo0, hi0, words);
+            decode_word<FMT>(cw[1], lo1, hi1, words + 16);
+          }
+          if (!__all_sync(0xffffffffu, slot_free) &&
+              !wait_bar_warp(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t dst = a_col + as * (kMT * kSlotCols);
+          tmem_st32(dst, words);
+          // hand the slot to the MMA warp once the stores have landed
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          mbar_arrive_if(&sh->full_a[as], lane == 0);
         }
-        if (!__all_sync(0xffffffffu, slot_free) &&
-            !wait_bar_warp(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t dst = a_col + as * (kMT * kSlotCols);
-        tmem_st32(dst, words);
-        // hand the slot to the MMA warp once the stores have landed
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        mbar_arrive_if(&sh->full_a[as], lane == 0);
-      }
+      };
+      // the code bytes of every step of this block start at the same offset
+      // mod 8 (8i and 4i*2 are multiples of 8): one warp-uniform choice
+      const int ocode = __shfl_sync(0xffffffffu, off + Fmt<FMT>::kCodeOff, 0) & 7;
+      if (!uniform8) steps(std::integral_constant<int, 0>{});
+      else if (ocode < 4) steps(std::integral_constant<int, 1>{});
+      else steps(std::integral_constant<int, 2>{});
       __syncwarp();
       mbar_arrive_if(&sh->empty_raw[rs], lane == 0);
       if (++kb == nblk) {
@@ -750,7 +808,6 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
         const int s = c % kRawStages;
         ok = wait_bar_warp(&sh->empty_raw[s], ((c / kRawStages) & 1) ^ 1, sh, w.status);
         if (!ok) break;
-        uint8_t* stage = raw_base + s * raw_stage_bytes<FMT>() + tile * 128 * PITCH;
         const uint8_t* blk0 = row0 + (size_t)kb * BB;
         if constexpr (GATEUP) {
           // rows 552+ bytes apart: lane = row, the lane copies the 16-byte
@@ -760,7 +817,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
             const int rr = rr0 + lane;
             const uintptr_t b0 = reinterpret_cast<uintptr_t>(blk0) + (uint32_t)rr * (uint32_t)rowbytes;
             const uintptr_t a0 = b0 & ~(uintptr_t)15;
-            uint8_t* dst = stage + rr * PITCH;
+            uint8_t* dst = raw_base + s * raw_stage_bytes<FMT>() + raw_row_offset<FMT>(tile, rr);
             if (rr < valid) {
 #pragma unroll
               for (int ch = 0; ch < CHUNKS; ++ch)
@@ -776,7 +833,8 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
             const uintptr_t b0 = reinterpret_cast<uintptr_t>(blk0) + (uint32_t)row * (uint32_t)rowbytes;
             const uintptr_t a0 = (b0 & ~(uintptr_t)15) + 16 * ch;
             if (row < valid && a0 < b0 + BB)
-              cp_async16(stage + row * PITCH + ch * 16, reinterpret_cast<const void*>(a0));
+              cp_async16(raw_base + s * raw_stage_bytes<FMT>() + raw_row_offset<FMT>(tile, row) + ch * 16,
+                         reinterpret_cast<const void*>(a0));
           }
         }
         cp_async_mbar_arrive(&sh->full_raw[s]);

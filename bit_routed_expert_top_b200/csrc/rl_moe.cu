@@ -9,11 +9,14 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
+#include <algorithm>
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "route_group.cuh"
+#include "small_t.cuh"
 
 namespace {
 
@@ -90,6 +93,7 @@ constexpr int kLaunchesPerCall = 6;
 // tensor cores, 1: CUDA cores), the limit of every bounded device wait, and
 // the RL_DEBUG_* fault bits.  Read once per call into its Dims.
 std::atomic<int> g_gemm{0};
+std::atomic<int> g_path{0};   // 0: small chunks take the decode-regime path, 1: always the prefill path
 std::atomic<long long> g_wait_cycles{rl::kDefaultWaitCycles};
 std::atomic<int> g_fault{0};
 
@@ -236,6 +240,57 @@ void launch_route(const float* logits, const rl::Dims& d, const rl::Work& w, cud
   else rl::route_kernel<32><<<grid, 256, 0, s>>>(logits, d, w);
 }
 
+// ---- decode regime (chunks of at most rl::small::kMaxPairs pairs) ----------
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+// The two-launch path applies when the chunk is small and the shapes fit its
+// lane mapping: whole 256-value blocks, a power-of-two number of blocks per
+// row (lanes of a row in a warp), k * (blocks per down row) lanes per column,
+// and room for h in fp32 where the prefill path keeps h and o.
+bool small_path_fits(const rl::Dims& d, const Layout& L) {
+  if (g_path.load(std::memory_order_relaxed) != 0) return false;
+  if (d.P > rl::small::kMaxPairs || d.k > 32) return false;
+  if (d.H % rl::kBlockVals || d.I % rl::kBlockVals) return false;
+  if (!is_pow2(d.nbH) || d.nbH > 32 || !is_pow2(d.nbI) || d.k * d.nbI > 32) return false;
+  return L.h16 + (size_t)d.P * d.I * 4 <= L.total;
+}
+
+template <int FMT, int PER>
+cudaError_t launch_gateup_small(const void* x, const float* logits, const rl::Dims& d, const rl::Work& w,
+                                const rl::ExpertTable& tab, float* h32, cudaStream_t s) {
+  const int rows_c = 4 * (32 / d.nbH);
+  const size_t smem = (size_t)d.nbH * rl::small::kSlice * sizeof(float);
+  rl::small::gateup_small_kernel<FMT, PER><<<dim3(d.P, (d.I + rows_c - 1) / rows_c), rl::small::kThreads, smem, s>>>(
+      static_cast<const uint16_t*>(x), logits, d, w, tab, h32);
+  return cudaGetLastError();
+}
+
+template <int FMT>
+int launch_small(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
+                 const rl::Work& w, float* h32, float* y, cudaStream_t s) {
+  const bool prof = g_prof.load(std::memory_order_relaxed);
+  mark(0, s);
+  mark(1, s);
+  mark(2, s);
+  const int per = (d.E + 31) / 32;
+  cudaError_t e;
+  if (per <= 1) e = launch_gateup_small<FMT, 1>(x, logits, d, w, tab, h32, s);
+  else if (per <= 2) e = launch_gateup_small<FMT, 2>(x, logits, d, w, tab, h32, s);
+  else if (per <= 4) e = launch_gateup_small<FMT, 4>(x, logits, d, w, tab, h32, s);
+  else if (per <= 8) e = launch_gateup_small<FMT, 8>(x, logits, d, w, tab, h32, s);
+  else if (per <= 16) e = launch_gateup_small<FMT, 16>(x, logits, d, w, tab, h32, s);
+  else e = launch_gateup_small<FMT, 32>(x, logits, d, w, tab, h32, s);
+  if (e != cudaSuccess) return cuda_fail(e, "gateup_small_kernel launch");
+  mark(3, s);
+  e = rl::launch_k(rl::small::down_combine_small_kernel<FMT>, dim3(d.T, (d.H + 7) / 8), dim3(rl::small::kThreads), 0,
+                   s, !prof, d, w, tab, static_cast<const float*>(h32), y);
+  if (e != cudaSuccess) return cuda_fail(e, "down_combine_small_kernel launch");
+  mark(4, s);
+  mark(5, s);
+  if (prof) g_ev_recorded = true;
+  return RL_OK;
+}
+
 template <int FMT>
 int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
                const rl::Work& w, float* y, cudaStream_t s) {
@@ -268,7 +323,8 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
   }
   mark(4, s);
   rl::launch_k(rl::combine_kernel, dim3(d.T, (d.H + 1023) / 1024), dim3(128), 0, s, pdl,
-               d, static_cast<const float*>(w.pw), static_cast<const __half*>(w.o16), y);
+               d, static_cast<const float*>(w.pw), static_cast<const int*>(w.pair_pos),
+               static_cast<const __half*>(w.o16), y);
   mark(5, s);
   if (prof) g_ev_recorded = true;
   const cudaError_t e = cudaGetLastError();
@@ -302,6 +358,12 @@ void* g_noalloc_addr[kMaxDevices] = {};
 }  // namespace
 
 extern "C" {
+
+// Error reporting for the other translation unit of the library (not in the
+// public header).
+__attribute__((visibility("hidden"))) int rl_moe_internal_fail(int code, const char* msg) {
+  return fail(code, "%s", msg);
+}
 
 size_t rl_moe_block_bytes(int fmt) {
   return fmt == RL_FMT_Q2 ? rl::kQ2Bytes : fmt == RL_FMT_Q1 ? rl::kQ1Bytes : 0;
@@ -341,6 +403,11 @@ int rl_moe_prefill_ws(const void* x, const float* router_logits, const void* con
   if (rc != RL_OK) return rc;
   const rl::Work w = carve(workspace, L);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (small_path_fits(d, L)) {
+    float* h32 = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.h16);
+    return fmt == RL_FMT_Q2 ? launch_small<RL_FMT_Q2>(x, router_logits, tab, d, w, h32, y, s)
+                            : launch_small<RL_FMT_Q1>(x, router_logits, tab, d, w, h32, y, s);
+  }
   return fmt == RL_FMT_Q2 ? launch_all<RL_FMT_Q2>(x, router_logits, tab, d, w, y, s)
                           : launch_all<RL_FMT_Q1>(x, router_logits, tab, d, w, y, s);
 }
@@ -425,6 +492,44 @@ int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx,
   return RL_OK;
 }
 
+int rl_moe_verify_bounded(rl_moe_cache* cache, const void* x, const float* router_logits, int T, int k,
+                          float* y, void* workspace, size_t ws_bytes, int* idx_host, void* stream) {
+  int fmt, H, I, E;
+  int rc = rl_moe_cache_shape(cache, &fmt, &H, &I, &E);
+  if (rc != RL_OK) return rc;
+  rl::Dims d;
+  Layout L;
+  rc = plan(fmt, T, H, I, E, k, &d, &L);
+  if (rc != RL_OK) return rc;
+  if (T == 0) return RL_OK;
+  if (!x || !router_logits || !y || !workspace)
+    return fail(RL_ERR_INVALID_ARG, "NULL x, router_logits, y or workspace");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(RL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < L.total)
+    return fail(RL_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, L.total);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // 1. the rows' router selections (the same exact top-k as the layer), read
+  //    back to the host
+  const rl::Work w = carve(workspace, L);
+  launch_route(router_logits, d, w, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "route_kernel launch");
+  std::vector<int> idx((size_t)d.P);
+  e = cudaMemcpyAsync(idx.data(), w.idx, idx.size() * sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the routing back");
+  if (idx_host) std::copy(idx.begin(), idx.end(), idx_host);
+  // 2. one prepare of the union of every row's experts
+  rc = rl_moe_cache_prepare(cache, idx.data(), d.P, stream);
+  if (rc != RL_OK) return rc;
+  // 3. the layer on the cache's slots (its routing picks exactly those experts)
+  std::vector<const void*> table((size_t)E);
+  rc = rl_moe_cache_table(cache, table.data(), E);
+  if (rc != RL_OK) return rc;
+  return rl_moe_prefill_ws(x, router_logits, table.data(), fmt, T, H, I, E, k, y, workspace, ws_bytes, stream);
+}
+
 int rl_moe_check_status(void* workspace, void* stream, unsigned* bits_out) {
   if (!workspace) return fail(RL_ERR_INVALID_ARG, "NULL workspace");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -473,6 +578,14 @@ const char* rl_moe_profile_stage_name(int i) {
 }
 
 int rl_moe_launches_per_call(void) { return kLaunchesPerCall; }
+
+// 0: chunks of at most 64 pairs take the two-launch decode-regime path where
+// their shapes fit it (the default); 1: every chunk takes the prefill path.
+int rl_moe_debug_set_path(int which) {
+  if (which != 0 && which != 1) return fail(RL_ERR_INVALID_ARG, "path %d", which);
+  g_path = which;
+  return RL_OK;
+}
 
 int rl_moe_debug_set_gemm(int which) {
   if (which != 0 && which != 1) return fail(RL_ERR_INVALID_ARG, "gemm %d", which);

@@ -360,11 +360,12 @@ __global__ void __launch_bounds__(256) place_pairs_kernel(const uint16_t* __rest
 }
 
 // Step 5: y[t, c] = sum_j p_{t,j} o_{t*k+j}[c], added in selection order j.
-// 8 columns per thread (16-byte loads), slots loaded four at a time ahead of
-// their fp32 fused multiply-adds, which run in j order.
+// o is in grouped order: pair t*k+j's row is pair_pos[t*k+j].  8 columns per
+// thread (16-byte loads), rows loaded four at a time ahead of their fp32 fused
+// multiply-adds, which run in j order.
 __global__ void __launch_bounds__(256)
-combine_kernel(Dims d, const float* __restrict__ pw, const __half* __restrict__ o16,
-               float* __restrict__ y) {
+combine_kernel(Dims d, const float* __restrict__ pw, const int* __restrict__ pair_pos,
+               const __half* __restrict__ o16, float* __restrict__ y) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;
@@ -381,7 +382,8 @@ combine_kernel(Dims d, const float* __restrict__ pw, const __half* __restrict__ 
 #pragma unroll
     for (int jj = 0; jj < kJ; ++jj) {
       if (j0 + jj < d.k) {
-        raw[jj] = __ldg(reinterpret_cast<const uint4*>(o16 + (base + j0 + jj) * d.H + c));
+        const int row = __ldg(pair_pos + base + j0 + jj);
+        raw[jj] = __ldg(reinterpret_cast<const uint4*>(o16 + (size_t)row * d.H + c));
         p[jj] = __ldg(pw + base + j0 + jj);
       }
     }

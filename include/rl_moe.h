@@ -177,6 +177,65 @@ int rl_moe_route(const float* router_logits, int T, int E, int k, int* topk_idx,
                  float* topk_w, int* offsets, int* pair_list, int* pair_pos,
                  void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Bounded expert cache ("Red Lite dev72 - bounded verify, profiling",
+ * section 1: a verify step on a machine that cannot hold every expert makes
+ * the union of its rows' experts resident in one prepare, so that loading
+ * one row's experts cannot evict another row's, and gives each row a plan of
+ * its own experts in its own selection order; routing stays exact).
+ * A cache holds up to `slots` of the E expert blobs in one device pool
+ * (256-byte aligned slots), filled from the caller's host copies.
+ */
+typedef struct rl_moe_cache rl_moe_cache;
+
+/* Pool in host memory instead of device memory: the bookkeeping alone, for
+ * tests without a GPU (such a cache has no device table). */
+#define RL_CACHE_HOST_POOL 0x1
+
+/* Creates a cache of `slots` (1..E) experts of format fmt and shape (H, I).
+ * host_blobs: HOST array of E host pointers to the experts' blobs
+ * (rl_moe_expert_bytes each), which must stay valid and unchanged while the
+ * cache lives; pinned host memory makes the copies asynchronous.  Allocates
+ * the pool with cudaMalloc (device current at the call). */
+int rl_moe_cache_create(int fmt, int H, int I, int E, int slots,
+                        const void* const* host_blobs, int flags, rl_moe_cache** out);
+/* Frees the pool (cudaFree) and the handle; NULL is a no-op. */
+int rl_moe_cache_destroy(rl_moe_cache* cache);
+/* Makes every expert of experts[0..n) resident (the union; repeats allowed):
+ * missing ones are copied host -> device on `stream` into empty slots, else
+ * into the least recently used slots whose experts are not in the union.
+ * RL_ERR_UNSUPPORTED when the union has more experts than the cache has
+ * slots.  A slot changes only inside a prepare, so work ordered on `stream`
+ * after a prepare sees its slots until the next prepare on that stream. */
+int rl_moe_cache_prepare(rl_moe_cache* cache, const int* experts, int n, void* stream);
+/* Host array of E device pointers for rl_moe_prefill[_ws]: resident experts
+ * at their slots, the others at slot 0 (a call whose routing picks only
+ * resident experts never reads them). */
+int rl_moe_cache_table(rl_moe_cache* cache, const void** table, int E);
+/* Per-row plans: for rows t < T with k experts each (idx, [T, k] host, in
+ * each row's selection order), plans[t*k + j] = the slot address of expert
+ * idx[t*k + j].  RL_ERR_INVALID_ARG if one of them is not resident. */
+int rl_moe_cache_plan(rl_moe_cache* cache, const int* idx, int T, int k, const void** plans);
+/* The cache's format and shape. */
+int rl_moe_cache_shape(rl_moe_cache* cache, int* fmt, int* H, int* I, int* E);
+/* *slot = the slot holding `expert`, or -1 when it is not resident. */
+int rl_moe_cache_slot_of(rl_moe_cache* cache, int expert, int* slot);
+/* Counters since creation: out4 = {hits, misses, bytes copied, evictions}. */
+int rl_moe_cache_stats(rl_moe_cache* cache, long long* out4);
+
+/*
+ * One bounded verify / decode step on a cache: the T rows' router selections
+ * (the layer's own exact top-k, on the device, read back to the host, which
+ * synchronizes `stream`), one prepare of their union, then rl_moe_prefill_ws
+ * on the cache's table.  x, router_logits, y and the workspace as for
+ * rl_moe_prefill_ws (shape and format from the cache); idx_host (may be NULL)
+ * receives the [T, k] selections.  y equals the layer with every expert
+ * resident, bit for bit.
+ */
+int rl_moe_verify_bounded(rl_moe_cache* cache, const void* x, const float* router_logits, int T,
+                          int k, float* y, void* workspace, size_t ws_bytes, int* idx_host,
+                          void* stream);
+
 /* Synchronizes `stream`, reads and clears the device status word of
  * `workspace`: the RL_DEV_* bits of the latest call on it (each call clears
  * the word when it starts).  Returns RL_OK, or RL_ERR_DEVICE_STATUS with the

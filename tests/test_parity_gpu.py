@@ -26,8 +26,10 @@ from bit_routed_expert_top_b200 import api  # noqa: E402
 @pytest.fixture(autouse=True)
 def _tc_default():
     api.debug_set_gemm("tc")
+    api.debug_set_path("auto")
     yield
     api.debug_set_gemm("tc")
+    api.debug_set_path("auto")
 
 
 def run_prefill(inp, ws=None):
@@ -137,6 +139,53 @@ def test_small_chunks_every_output(wl):
     Hh.assert_y_close(y, ref["y"], wl.name)
 
 
+DECODE_REGIME = [
+    synth.WORKLOADS[1],                                              # verify2: T=2, 512 experts, top-10
+    synth.Workload("dr_t1", 1, 2048, 512, 512, 10, synth.FMT_Q2),    # one-token decode step
+    synth.Workload("dr_t1_q1", 1, 2048, 512, 512, 10, synth.FMT_Q1),
+    synth.Workload("dr_t4_q1", 4, 1024, 512, 64, 8, synth.FMT_Q1),  # 4 blocks per gate/up row
+    synth.Workload("dr_t6", 6, 512, 256, 48, 10, synth.FMT_Q2),     # P = 60
+    synth.Workload("dr_k32", 2, 256, 256, 64, 32, synth.FMT_Q2),    # k * blocks per down row = 32 lanes
+    synth.Workload("dr_e1024", 2, 512, 256, 1024, 8, synth.FMT_Q1), # 32 logits per lane
+]
+
+
+@pytest.mark.parametrize("wl", DECODE_REGIME, ids=lambda w: w.name)
+def test_decode_regime_every_output_and_against_the_prefill_path(wl):
+    """Chunks of at most 64 pairs whose shapes fit it take the two-launch
+    decode-regime path: every output against the oracle, the routing it
+    publishes bit for bit, and the same inputs forced through the six-launch
+    prefill path (both within the layer's tolerance of the oracle)."""
+    inp = synth.make_inputs(wl, seed=11 + sum(wl.name.encode()))
+    ref = full_oracle(inp)
+    y_small, ws = run_prefill(inp)
+    Hh.assert_y_close(y_small, ref["y"], wl.name + " (decode regime)")
+    P = wl.T * wl.k
+    raw = ws.cpu().numpy()
+    # idx and p follow the 256-byte status piece of the workspace
+    idx = raw[256:256 + 4 * P].view(np.int32).reshape(wl.T, wl.k)
+    off_p = 256 + (4 * P + 255) // 256 * 256
+    pw = raw[off_p:off_p + 4 * P].view(np.float32).reshape(wl.T, wl.k)
+    np.testing.assert_array_equal(idx, ref["idx"])
+    np.testing.assert_allclose(pw, ref["p"], rtol=0, atol=Hh.P_ATOL)
+    api.debug_set_path("prefill")
+    y_pre, _ = run_prefill(inp)
+    Hh.assert_y_close(y_pre, ref["y"], wl.name + " (prefill path)")
+
+
+def test_decode_regime_ties_in_the_router():
+    """Exact ties (and -0.0 against +0.0) at the k / k+1 boundary and inside
+    the top k on the decode-regime path: the lower expert index wins, as in
+    the oracle."""
+    wl = synth.Workload("dr_ties", 2, 512, 256, 40, 6, synth.FMT_Q2)
+    inp = synth.make_inputs(wl, seed=3)
+    vals = np.array([-1.0, -0.0, 0.0, 0.5, 1.0], dtype=np.float32)
+    inp.logits[:] = vals[np.random.default_rng(5).integers(0, len(vals), inp.logits.shape)]
+    ref = full_oracle(inp)
+    y, _ = run_prefill(inp)
+    Hh.assert_y_close(y, ref["y"], "decode regime with ties")
+
+
 def test_layer_heavy_expert_many_n_tiles():
     """One expert takes every token (n_e = T > one N tile), most experts
     get no pair at all."""
@@ -160,9 +209,11 @@ def test_layer_zero_down_is_zero():
     assert np.all(y == 0.0)
 
 
-def workspace_h_o(ws, wl):
-    """h (grouped order, K-permutation undone) and o (pair-id order) of the
-    last call, read from the last two pieces of the workspace."""
+def workspace_h_o(ws, wl, pair_pos):
+    """h (grouped order, K-permutation undone) and o (put in pair-id order
+    with the oracle's inverse list, which the routing tests check against the
+    library's bit for bit) of the last call, read from the last two pieces of
+    the workspace."""
     n = api.rl_moe_workspace_bytes(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k)
     P = wl.T * wl.k
     raw = ws.cpu().numpy()
@@ -172,7 +223,7 @@ def workspace_h_o(ws, wl):
     h_off = o_off - ((h_bytes + 255) // 256 * 256)
     h = raw[h_off:h_off + h_bytes].view(np.float16).reshape(P, wl.I).astype(np.float64)
     o = raw[o_off:o_off + o_bytes].view(np.float16).reshape(P, wl.H).astype(np.float64)
-    return Hh.unpermute_k(h, wl.fmt), o
+    return Hh.unpermute_k(h, wl.fmt), o[np.asarray(pair_pos)]
 
 
 def test_intermediates_h_and_o_tiny():
@@ -180,7 +231,7 @@ def test_intermediates_h_and_o_tiny():
     wl = inp.wl
     y, ws = run_prefill(inp)
     ref = full_oracle(inp)
-    h, o = workspace_h_o(ws, wl)
+    h, o = workspace_h_o(ws, wl, ref["pair_pos"])
     rel_h = np.linalg.norm(h - ref["h"]) / np.linalg.norm(ref["h"])
     rel_o = np.linalg.norm(o - ref["o"]) / np.linalg.norm(ref["o"])
     assert rel_h < 2e-3, rel_h
@@ -256,7 +307,7 @@ def test_edge_blocks_every_output(wl):
     y, ws = run_prefill(inp)
     ref = full_oracle(inp)
     Hh.assert_y_close(y, ref["y"], wl.name)
-    h, o = workspace_h_o(ws, wl)
+    h, o = workspace_h_o(ws, wl, ref["pair_pos"])
     assert Hh.y_errors(h, ref["h"])[0] < 2e-3
     assert Hh.y_errors(o, ref["o"])[0] < 2e-3
 
