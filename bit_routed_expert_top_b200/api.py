@@ -52,6 +52,7 @@ DEBUG_SIGNATURES = {
     "rl_moe_debug_set_gemm": (_i, [_i]),
     "rl_moe_debug_set_fault": (_i, [_i, ctypes.c_longlong]),
     "rl_moe_debug_set_path": (_i, [_i]),
+    "rl_moe_debug_set_raw_tma": (_i, [_i]),
 }
 RL_DEV_UNIT_OVERFLOW = 0x1
 RL_DEV_WAIT_TIMEOUT = 0x2
@@ -330,6 +331,12 @@ def debug_set_path(which: str):
     path where their shapes fit it; the default) or 'prefill' (always the
     six-launch prefill path)."""
     _check(load().rl_moe_debug_set_path({"auto": 0, "prefill": 1}[which]))
+
+
+def debug_set_raw_tma(on: bool):
+    """Gate/up raw blocks by TMA when the experts sit at one stride (the
+    default) or always by per-lane cp.async."""
+    _check(load().rl_moe_debug_set_raw_tma(1 if on else 0))
 
 
 def debug_set_gemm(which: str):

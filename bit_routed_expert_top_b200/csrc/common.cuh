@@ -89,6 +89,8 @@ struct Dims {
   int nt_gu;      // max pairs per gate/up work unit
   int nt_dn;      // max pairs per down work unit
   int max_units_gu, max_units_dn;
+  int raw_tma;            // gate/up raw blocks by TMA from one 3-D map over all experts
+  long long expert_stride;  // bytes between consecutive experts' blobs when raw_tma
   long long wait_cycles;  // limit of every bounded device wait, in SM clock cycles
   int debug_fault;        // RL_DEBUG_* bits (0 on every normal call)
 };

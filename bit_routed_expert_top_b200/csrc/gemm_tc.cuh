@@ -65,6 +65,14 @@ namespace tc {
 #ifndef RL_TC_DEC_PHASES
 #define RL_TC_DEC_PHASES 2
 #endif
+// Back-off (ns of __nanosleep between polls) of the waits of the raw-fetch
+// warps and of the MMA warp; 0 polls without sleeping.
+#ifndef RL_TC_FETCH_SLEEP_NS
+#define RL_TC_FETCH_SLEEP_NS 0
+#endif
+#ifndef RL_TC_MMA_SLEEP_NS
+#define RL_TC_MMA_SLEEP_NS 0
+#endif
 constexpr int kNT = RL_TC_NT;    // max pairs per unit = accumulator columns per tile
 constexpr int kNtGu = kNT;       // gate/up unit size in pairs
 constexpr int kNtDn = kNT;       // down unit size in pairs
@@ -282,17 +290,17 @@ struct Shared {
 };
 static_assert(sizeof(Shared) + 16 <= kSharedBytes, "shared-memory control block");
 
-// Bounded wait.  Roles whose waits are long (epilogue, B gather) pass
-// sleepy=true and back off with nanosleep, leaving issue slots to the
-// decoder warps on the same scheduler; the MMA and decoder warps spin.
+// Bounded wait.  Roles whose waits are long (epilogue, B operand) pass a
+// back-off of sleep_ns and sleep between polls, leaving issue slots to the
+// decoder warps on the same scheduler; sleep_ns = 0 polls continuously.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared* sh, unsigned* status,
-                                         bool sleepy = false) {
+                                         uint32_t sleep_ns = 0) {
   const uint32_t addr = smem_addr(bar);
   long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(addr, parity)) return true;
-    if (sleepy) __nanosleep(256);
-    if (sleepy || (it & 15u) == 15u) {
+    if (sleep_ns) __nanosleep(sleep_ns);
+    if (sleep_ns || (it & 15u) == 15u) {
       if (*(volatile int*)&sh->abort_flag) return false;
       const long long now = clock64();
       if (t0 == 0) {
@@ -307,10 +315,11 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared*
 }
 // Warp-uniform variant: every lane waits, the result is agreed with a vote.
 __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, Shared* sh, unsigned* status,
-                                              bool sleepy = false) {
+                                              uint32_t sleep_ns = 0) {
   if (__all_sync(0xffffffffu, mbar_try_wait(smem_addr(bar), parity))) return true;
-  return __all_sync(0xffffffffu, wait_bar(bar, parity, sh, status, sleepy));
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, sh, status, sleep_ns));
 }
+constexpr uint32_t kSleepNs = 256;             // epilogue and B-operand waits
 // Bounded wait that does not give up on the abort flag: used where this
 // thread's own asynchronous operations must have finished before the CTA may
 // leave (MMAs reading TMEM, TMA writes into shared memory).
@@ -491,9 +500,25 @@ __device__ __forceinline__ const uint8_t* tile_row(const Dims& d, const uint8_t*
   return mat + (size_t)R * rowbytes;
 }
 
+// TMA: 3D tile load (x, y, z) into shared memory, completion counted in
+// bytes on an mbarrier (one CTA, plain load).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Bytes of one raw stage loaded by TMA (gate/up, d.raw_tma): both tiles'
+// even and odd rows, a box of kPitch bytes x 64 row pairs each.
+template <int FMT>
+__host__ __device__ constexpr int raw_tma_stage_bytes() { return kMT * 2 * 64 * Raw<FMT>::kPitch; }
+
 template <int FMT, bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUtensorMap bmap) {
+decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUtensorMap bmap,
+                   const __grid_constant__ CUtensorMap rawmap) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -530,7 +555,9 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRawStages; ++s) {
-      mbar_init(&sh->full_raw[s], kMT * 32); // fetch warps x 32 lanes (cp.async arrivals)
+      // TMA fetch: one arrival with the byte count; cp.async fetch: every
+      // lane of both fetch warps
+      mbar_init(&sh->full_raw[s], GATEUP && d.raw_tma ? 1 : kMT * 32);
       mbar_init(&sh->empty_raw[s], kDecWarps);  // every decoder warp releases every block
     }
     for (int s = 0; s < kBStages; ++s) {
@@ -585,20 +612,21 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       const int npad = max(16, (cnt + 15) & ~15);
       const uint32_t idesc = idesc_f16(128, npad);
       const int buf = ui & 1;
-      if (ui >= kAccBufs) ok = wait_bar_warp(&sh->acc_empty[buf], ((ui / kAccBufs) - 1) & 1, sh, w.status);
+      if (ui >= kAccBufs)
+        ok = wait_bar_warp(&sh->acc_empty[buf], ((ui / kAccBufs) - 1) & 1, sh, w.status, RL_TC_MMA_SLEEP_NS);
       tc_fence_after();
       const uint32_t acc0 = tmem + buf * (kMT * kNT);
       for (int st = 0; st < nstep && ok; st += kStepsPerB) {
-        if (!wait_bar_warp(&sh->full_b[bs], bph, sh, w.status)) { ok = false; break; }
+        if (!wait_bar_warp(&sh->full_b[bs], bph, sh, w.status, RL_TC_MMA_SLEEP_NS)) { ok = false; break; }
         const uint64_t bd = bdesc0 + (uint64_t)((bs * kBStageBytes) >> 4);
         // step st: K block 0 of the stage
-        if (!wait_bar_warp(&sh->full_a[as], aph, sh, w.status)) { ok = false; break; }
+        if (!wait_bar_warp(&sh->full_a[as], aph, sh, w.status, RL_TC_MMA_SLEEP_NS)) { ok = false; break; }
         tc_fence_after();
         mma_step2x(acc0, a_base + as * (kMT * kSlotCols), bd, idesc, st != 0, 2 * st + 1 < nsub, &sh->empty_a[as]);
         if (++as == kRing) { as = 0; aph ^= 1; }
         // step st + 1: K block 1 of the stage
         if (st + 1 < nstep) {
-          if (!wait_bar_warp(&sh->full_a[as], aph, sh, w.status)) { ok = false; break; }
+          if (!wait_bar_warp(&sh->full_a[as], aph, sh, w.status, RL_TC_MMA_SLEEP_NS)) { ok = false; break; }
           tc_fence_after();
           mma_step2x(acc0, a_base + as * (kMT * kSlotCols), bd + (kBBlockBytes >> 4), idesc, 1u,
                      2 * st + 3 < nsub, &sh->empty_a[as]);
@@ -623,7 +651,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       const int n0 = unit_at(ui).z;
       for (int kc = 0; kc < nbchunk && ok; ++kc, ++b_it) {
         const int s = b_it % kBStages;
-        ok = wait_bar_warp(&sh->empty_b[s], ((b_it / kBStages) & 1) ^ 1, sh, w.status, true);
+        ok = wait_bar_warp(&sh->empty_b[s], ((b_it / kBStages) & 1) ^ 1, sh, w.status, kSleepNs);
         if (!ok) break;
         uint8_t* stage = b_base + s * kBStageBytes;
         if (lane == 0) mbar_arrive_expect_tx(&sh->full_b[s], (uint32_t)kBStageBytes);
@@ -649,7 +677,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       const int4 un = unit_at(ui);
       const int buf = ui & 1;
       const int cnt = un.w, n0 = un.z;
-      if (!wait_bar_warp(&sh->acc_full[buf], (ui / kAccBufs) & 1, sh, w.status, true)) break;
+      if (!wait_bar_warp(&sh->acc_full[buf], (ui / kAccBufs) & 1, sh, w.status, kSleepNs)) break;
       tc_fence_after();
       const uint32_t acc0 = tmem + lane_addr + buf * (kMT * kNT);
       for (int cc = 0; cc * 16 < cnt; ++cc) {
@@ -792,10 +820,54 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     }
   } else {
     // ----------------------------------------------------- raw fetch -----
+    const int tile = warp - kFetchWarp0;
+    if (GATEUP && d.raw_tma) {
+      // One 3-D tensor map covers every expert's gate/up rows as row pairs
+      // (x: byte in the pair, y: pair, z: expert): for a K block, tile t's
+      // even rows and odd rows are two boxes of kPitch bytes x 64 pairs whose
+      // x starts at the block's 16-byte aligned offset in the first / second
+      // row of a pair; they land in the parity-split row layout the
+      // decoders read (block at the same offset mod 16 as with cp.async).
+      if (tile != 0) {
+        // the second fetch warp has nothing to do on this path
+      } else {
+        uint32_t c = 0;
+        bool ok = true;
+        for (int ui = 0; ui < my_units && ok; ++ui) {
+          const int4 un = unit_at(ui);
+          const int z = un.x;
+          for (int kb = 0; kb < nblk && ok; ++kb, ++c) {
+            const int s = c % kRawStages;
+            ok = wait_bar_warp(&sh->empty_raw[s], ((c / kRawStages) & 1) ^ 1, sh, w.status, RL_TC_FETCH_SLEEP_NS);
+            if (!ok) break;
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&sh->full_raw[s], (uint32_t)raw_tma_stage_bytes<FMT>());
+              uint8_t* st0 = raw_base + s * raw_stage_bytes<FMT>();
+              const int bo = kb * BB;                          // block offset in a row
+#pragma unroll
+              for (int t = 0; t < kMT; ++t) {
+                const int y = t * (d.I / 2) + un.y * 64;       // first pair of the slab
+#pragma unroll
+                for (int par = 0; par < 2; ++par) {
+                  const int x = (par * (int)rowbytes + bo) & ~15;
+                  tma_load_3d(st0 + raw_row_offset<FMT>(t, par), &rawmap, x, y, z, &sh->full_raw[s]);
+                }
+              }
+            }
+            __syncwarp();
+          }
+        }
+        // after an abort, the boxes this warp requested land before the CTA
+        // leaves: wait for the last load of every stage
+        if (!ok) {
+          for (uint32_t i = c > (uint32_t)kRawStages ? c - kRawStages : 0u; i < c; ++i)
+            __all_sync(0xffffffffu, wait_bar_own(&sh->full_raw[i % kRawStages], (i / kRawStages) & 1, sh, w.status));
+        }
+      }
+    } else {
     // Warp kFetchWarp0 + t copies M tile t's rows.  A row's block starts at
     // an arbitrary byte: the 16-byte chunks that hold it are copied, and the
     // decoders find the block at the start address's offset mod 16.
-    const int tile = warp - kFetchWarp0;
     constexpr int kCopies = 128 * CHUNKS / 32;  // cp.async per lane per block
     bool ok = true;
     int c = 0;
@@ -806,7 +878,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       const int valid = min(128, rows_total - R0);   // rows of this tile inside the matrix
       for (int kb = 0; kb < nblk; ++kb, ++c) {
         const int s = c % kRawStages;
-        ok = wait_bar_warp(&sh->empty_raw[s], ((c / kRawStages) & 1) ^ 1, sh, w.status);
+        ok = wait_bar_warp(&sh->empty_raw[s], ((c / kRawStages) & 1) ^ 1, sh, w.status, RL_TC_FETCH_SLEEP_NS);
         if (!ok) break;
         const uint8_t* blk0 = row0 + (size_t)kb * BB;
         if constexpr (GATEUP) {
@@ -842,6 +914,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     }
     // copies still in flight after an abort land before the CTA leaves
     asm volatile("cp.async.wait_all;" ::: "memory");
+    }
   }
 
   tc_fence_before();

@@ -63,7 +63,7 @@ int num_sms(int dev) {
 // set once per device (setting it twice from racing threads is harmless).
 template <int FMT, bool GATEUP>
 int launch_decode_gemm(const rl::Dims& d, const rl::Work& w, const rl::ExpertTable& tab, const CUtensorMap& bmap,
-                       cudaStream_t s, bool pdl) {
+                       const CUtensorMap& rawmap, cudaStream_t s, bool pdl) {
   static std::atomic<unsigned long long> configured{0};
   constexpr int smem = rl::tc::smem_bytes<FMT>();
   const int dev = current_device();
@@ -77,7 +77,7 @@ int launch_decode_gemm(const rl::Dims& d, const rl::Work& w, const rl::ExpertTab
   const int maxu = GATEUP ? d.max_units_gu : d.max_units_dn;
   const int sms = num_sms(dev);
   const cudaError_t e = rl::launch_k(rl::tc::decode_gemm_kernel<FMT, GATEUP>, dim3(maxu < sms ? maxu : sms),
-                                     dim3(rl::tc::kThreads), smem, s, pdl, d, w, tab, bmap);
+                                     dim3(rl::tc::kThreads), smem, s, pdl, d, w, tab, bmap, rawmap);
   return e == cudaSuccess ? RL_OK : cuda_fail(e, "decode_gemm_kernel launch");
 }
 
@@ -93,7 +93,8 @@ constexpr int kLaunchesPerCall = 6;
 // tensor cores, 1: CUDA cores), the limit of every bounded device wait, and
 // the RL_DEBUG_* fault bits.  Read once per call into its Dims.
 std::atomic<int> g_gemm{0};
-std::atomic<int> g_path{0};   // 0: small chunks take the decode-regime path, 1: always the prefill path
+std::atomic<int> g_path{0};
+std::atomic<int> g_raw_tma{1};  // 1: gate/up raw blocks by TMA when the expert table allows it   // 0: small chunks take the decode-regime path, 1: always the prefill path
 std::atomic<long long> g_wait_cycles{rl::kDefaultWaitCycles};
 std::atomic<int> g_fault{0};
 
@@ -133,6 +134,8 @@ int plan(int fmt, int T, int H, int I, int E, int k, rl::Dims* d, Layout* L) {
   d->nt_dn = kNtDown;
   d->max_units_gu = d->slabs_gu * (E + (d->P + kNtGateUp - 1) / kNtGateUp);
   d->max_units_dn = d->groups_dn * (E + (d->P + kNtDown - 1) / kNtDown);
+  d->raw_tma = 0;
+  d->expert_stride = 0;
   d->wait_cycles = g_wait_cycles.load(std::memory_order_relaxed);
   d->debug_fault = g_fault.load(std::memory_order_relaxed);
   size_t o = 0;
@@ -227,6 +230,40 @@ int make_act_map(CUtensorMap* map, const void* base, int K, long long rows, int 
   return RL_OK;
 }
 
+// The gate/up raw blocks of every expert as one 3-D uint8 tensor: x = byte
+// in a pair of consecutive rows (2 * row bytes, a multiple of 16), y = row
+// pair (gate and up: I pairs), z = expert (experts `stride` bytes apart);
+// boxes of `pitch` bytes x 64 pairs.
+int make_raw_map(CUtensorMap* map, const void* base, long long pair_bytes, int pairs, int E, long long stride,
+                 int pitch) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(RL_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {(cuuint64_t)pair_bytes, (cuuint64_t)pairs, (cuuint64_t)E};
+  const cuuint64_t strides[2] = {(cuuint64_t)pair_bytes, (cuuint64_t)stride};
+  const cuuint32_t box[3] = {(cuuint32_t)pitch, 64u, 1u};
+  const cuuint32_t es[3] = {1u, 1u, 1u};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RL_ERR_CUDA, "cuTensorMapEncodeTiled (raw blocks) failed (CUresult %d)", (int)r);
+  return RL_OK;
+}
+
+// Whether the gate/up raw blocks can be fetched by TMA: the experts sit at
+// one positive stride (a multiple of 16), and a pair of gate/up rows is a
+// multiple of 16 bytes while a row is a multiple of 8 (so every lane's block
+// has the same offset mod 8, which the decoders' load path assumes too).
+long long uniform_expert_stride(const rl::ExpertTable& tab, const rl::Dims& d) {
+  const long long rowbytes = (long long)d.nbH * d.bb;
+  if ((2 * rowbytes) % 16 || rowbytes % 8) return 0;
+  if (d.E == 1) return (long long)((rl_moe_expert_bytes(d.fmt, d.H, d.I) + 15) / 16 * 16);
+  const long long s = (long long)(reinterpret_cast<uintptr_t>(tab.p[1]) - reinterpret_cast<uintptr_t>(tab.p[0]));
+  if (s <= 0 || s % 16) return 0;
+  for (int e = 2; e < d.E; ++e)
+    if ((long long)(reinterpret_cast<uintptr_t>(tab.p[e]) - reinterpret_cast<uintptr_t>(tab.p[0])) != s * e) return 0;
+  return s;
+}
+
 // Route: one CTA per 8 tokens over every byte column of the token bitmap;
 // values per lane = smallest power of two >= E/32.
 void launch_route(const float* logits, const rl::Dims& d, const rl::Work& w, cudaStream_t s) {
@@ -259,7 +296,7 @@ template <int FMT, int PER>
 cudaError_t launch_gateup_small(const void* x, const float* logits, const rl::Dims& d, const rl::Work& w,
                                 const rl::ExpertTable& tab, float* h32, cudaStream_t s) {
   const int rows_c = 4 * (32 / d.nbH);
-  const size_t smem = (size_t)d.nbH * rl::small::kSlice * sizeof(float);
+  const size_t smem = (size_t)d.nbH * rl::small::kSliceW * sizeof(__half2);
   rl::small::gateup_small_kernel<FMT, PER><<<dim3(d.P, (d.I + rows_c - 1) / rows_c), rl::small::kThreads, smem, s>>>(
       static_cast<const uint16_t*>(x), logits, d, w, tab, h32);
   return cudaGetLastError();
@@ -282,8 +319,10 @@ int launch_small(const void* x, const float* logits, const rl::ExpertTable& tab,
   else e = launch_gateup_small<FMT, 32>(x, logits, d, w, tab, h32, s);
   if (e != cudaSuccess) return cuda_fail(e, "gateup_small_kernel launch");
   mark(3, s);
-  e = rl::launch_k(rl::small::down_combine_small_kernel<FMT>, dim3(d.T, (d.H + 7) / 8), dim3(rl::small::kThreads), 0,
-                   s, !prof, d, w, tab, static_cast<const float*>(h32), y);
+  const size_t smem2 = (size_t)d.k * d.nbI * rl::small::kSliceW * sizeof(__half2);
+  e = rl::launch_k(rl::small::down_combine_small_kernel<FMT>,
+                   dim3(d.T, (d.H + rl::small::kDownCols - 1) / rl::small::kDownCols), dim3(rl::small::kThreads),
+                   smem2, s, !prof, d, w, tab, static_cast<const float*>(h32), y);
   if (e != cudaSuccess) return cuda_fail(e, "down_combine_small_kernel launch");
   mark(4, s);
   mark(5, s);
@@ -310,15 +349,24 @@ int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, c
     mark(3, s);
     rl::down_simt_kernel<FMT><<<d.max_units_dn, 256, 0, s>>>(d, w, tab);
   } else {
-    alignas(64) CUtensorMap xmap, hmap;
+    alignas(64) CUtensorMap xmap, hmap, rawmap;
     int rc = make_act_map(&xmap, w.x16, d.H, d.P, rl::tc::kNT);
     if (rc != RL_OK) return rc;
     rc = make_act_map(&hmap, w.h16, d.I, d.P, rl::tc::kNT);
     if (rc != RL_OK) return rc;
-    rc = launch_decode_gemm<FMT, true>(d, w, tab, xmap, s, pdl);
+    rl::Dims dg = d;
+    dg.expert_stride = g_raw_tma.load(std::memory_order_relaxed) ? uniform_expert_stride(tab, d) : 0;
+    dg.raw_tma = dg.expert_stride > 0;
+    if (dg.raw_tma) {
+      rc = make_raw_map(&rawmap, tab.p[0], 2LL * d.nbH * d.bb, d.I, d.E, dg.expert_stride, rl::tc::Raw<FMT>::kPitch);
+      if (rc != RL_OK) return rc;
+    } else {
+      rawmap = xmap;                                  // unused
+    }
+    rc = launch_decode_gemm<FMT, true>(dg, w, tab, xmap, rawmap, s, pdl);
     if (rc != RL_OK) return rc;
     mark(3, s);
-    rc = launch_decode_gemm<FMT, false>(d, w, tab, hmap, s, pdl);
+    rc = launch_decode_gemm<FMT, false>(d, w, tab, hmap, rawmap, s, pdl);
     if (rc != RL_OK) return rc;
   }
   mark(4, s);
@@ -584,6 +632,13 @@ int rl_moe_launches_per_call(void) { return kLaunchesPerCall; }
 int rl_moe_debug_set_path(int which) {
   if (which != 0 && which != 1) return fail(RL_ERR_INVALID_ARG, "path %d", which);
   g_path = which;
+  return RL_OK;
+}
+
+// 1 (default): gate/up raw blocks by TMA when the experts sit at one stride;
+// 0: always the per-lane cp.async fetch.
+int rl_moe_debug_set_raw_tma(int on) {
+  g_raw_tma = on != 0;
   return RL_OK;
 }
 

@@ -20,15 +20,18 @@
 //             nbH lanes of a row add up, and h = silu(g) * u is written in
 //             fp32 to the pair's row of h (in the K order of the down
 //             projection's decoder).  The CTAs of chunk 0 also write idx and p.
-//   launch 2  down_combine_small_kernel, grid (token, column chunk): warp =
-//             output column c of token t, lane (j, block) decodes one block
-//             of row c of expert idx[t,j]'s down matrix and dots it with
-//             h_{t,j}; the nbI lanes of a j add up, and lane 0 adds
-//             p_j * o_j over j = 0..k-1 in selection order into y[t, c].
+//   launch 2  down_combine_small_kernel, grid (token, 32-column chunk): the
+//             CTA stages the token's k rows of h in shared memory (fp16, as
+//             the prefill path rounds h); warp = 4 output columns in turn,
+//             lane (j, block) decodes one block of row c of expert idx[t,j]'s
+//             down matrix and dots it with h_{t,j}; the nbI lanes of a j add
+//             up, and lane 0 adds p_j * o_j over j = 0..k-1 in selection
+//             order into y[t, c].
 //
-// Weights are decoded exactly as on the prefill path (one fp16 rounding of
-// d(2s+1)c per weight); sums are fp32, h is kept in fp32.  Both kernels are
-// plain loads and arithmetic: no waits on other CTAs.
+// Weights, x and h are rounded to fp16 exactly as on the prefill path; the
+// products of one code word (16 values) are summed in fp16 pairs and these
+// partials in fp32.  Both kernels are plain loads and arithmetic: no waits
+// on other CTAs.
 #pragma once
 
 #include "common.cuh"
@@ -40,19 +43,12 @@ namespace small {
 
 constexpr int kMaxPairs = 64;     // chunks up to this many pairs take this path
 constexpr int kThreads = 256;     // 8 warps
-constexpr int kXPad = 2;          // fp32 pad per 256-value x slice (bank spread)
-constexpr int kSlice = kBlockVals + kXPad;
+constexpr int kSliceW = kBlockVals / 2 + 4;   // fp16x2 words per 256-value activation slice (+4: bank spread)
+constexpr int kDownCols = 32;     // output columns per CTA of launch 2 (4 per warp)
 
-// acc += a * b, two fp32 lanes at once (Blackwell packed FMA).
-__device__ __forceinline__ void ffma2(float2& acc, float2 a, float2 b) {
-  unsigned long long A = *reinterpret_cast<unsigned long long*>(&a);
-  unsigned long long B = *reinterpret_cast<unsigned long long*>(&b);
-  unsigned long long C = *reinterpret_cast<unsigned long long*>(&acc);
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(C) : "l"(A), "l"(B));
-  acc = *reinterpret_cast<float2*>(&C);
-}
-
-// 32 bits starting at byte address p (any alignment) of global memory.
+// 32 bits starting at byte address p (any alignment) of global memory.  Both
+// aligned words read hold at least one byte of the block (it is >= 38 bytes
+// long), so neither read leaves the 4-byte word around a valid byte.
 __device__ __forceinline__ uint32_t ldg_u32_at(const uint8_t* p) {
   const uintptr_t a = reinterpret_cast<uintptr_t>(p);
   const uint32_t* w = reinterpret_cast<const uint32_t*>(a & ~(uintptr_t)3);
@@ -60,11 +56,13 @@ __device__ __forceinline__ uint32_t ldg_u32_at(const uint8_t* p) {
 }
 
 // Dot product of one block (256 values of a row, at byte address blk) with
-// 256 fp32 activations xs stored in the decoder's K order (the order of
-// decode_word's fp16 halves).  Every weight is rounded once to fp16 exactly
-// as the tensor-core decoders round it.
+// 256 activations xs2 held as fp16x2 words in the decoder's K order (word w
+// = the two values decode_word puts in its output word w).  Every weight is
+// rounded once to fp16 exactly as the tensor-core decoders round it; the 16
+// products of a code word are summed in fp16x2 (8 fused multiply-adds per
+// half), each code word's partial then in fp32.
 template <int FMT>
-__device__ __forceinline__ float block_dot(const uint8_t* blk, const float* xs) {
+__device__ __forceinline__ float block_dot(const uint8_t* blk, const __half2* xs2) {
   constexpr int kCodeOff = Fmt<FMT>::kCodeOff;
   constexpr int G = Fmt<FMT>::kGroup;               // values per code word
   const uint32_t h0 = ldg_u32_at(blk), h1 = ldg_u32_at(blk + 4);
@@ -79,10 +77,10 @@ __device__ __forceinline__ float block_dot(const uint8_t* blk, const float* xs) 
   uint32_t raw[kWords + 1];
 #pragma unroll
   for (int i = 0; i < kWords; ++i) raw[i] = __ldg(cw + i);
-  // the word after the last is needed (and inside the block) only when the
-  // code bytes do not start on a word boundary
+  // the word after the last is needed (and holds the block's last byte) only
+  // when the code bytes do not start on a word boundary
   raw[kWords] = sh ? __ldg(cw + kWords) : 0u;
-  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+  float total = 0.f;
 #pragma unroll
   for (int sb = 0; sb < kBlockVals / kSubVals; ++sb) {
     uint32_t lo, hi;
@@ -94,25 +92,35 @@ __device__ __forceinline__ float block_dot(const uint8_t* blk, const float* xs) 
       const uint32_t word = __funnelshift_r(raw[g], raw[g + 1], sh);
       uint32_t out[G / 2];
       tc::decode_word<FMT>(word, lo, hi, out);
-      const float2* x2 = reinterpret_cast<const float2*>(xs + g * G);
+      const uint4* x4 = reinterpret_cast<const uint4*>(xs2 + g * (G / 2));
 #pragma unroll
-      for (int i = 0; i < G / 2; ++i) {
-        const float2 w2 = __half22float2(*reinterpret_cast<const __half2*>(&out[i]));
-        ffma2((i & 1) ? acc1 : acc0, w2, x2[i]);
+      for (int h8 = 0; h8 < G / 16; ++h8) {          // 8 words (16 values) per fp16 partial
+        __half2 acc = __float2half2_rn(0.f);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const uint4 xv = x4[h8 * 2 + q];
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            acc = __hfma2(*reinterpret_cast<const __half2*>(&out[h8 * 8 + q * 4 + i]),
+                          *reinterpret_cast<const __half2*>(&xw[i]), acc);
+        }
+        const float2 f = __half22float2(acc);
+        total += f.x + f.y;
       }
     }
   }
-  return (acc0.x + acc0.y) + (acc1.x + acc1.y);
+  return total;
 }
 
 // Launch 1.  grid (P, ceil(I / (4 * 32 / nbH))), 256 threads; PER as in
-// route_kernel; dynamic shared memory: nbH * kSlice floats (x_t).
+// route_kernel; dynamic shared memory: nbH * kSliceW fp16x2 words (x_t).
 template <int FMT, int PER>
 __global__ void __launch_bounds__(kThreads)
 gateup_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ logits, Dims d, Work w,
                     ExpertTable tab, float* __restrict__ h32) {
   pdl_trigger();
-  extern __shared__ __align__(16) float xs[];       // [nbH][kSlice]
+  extern __shared__ __align__(16) __half2 xs2[];    // [nbH][kSliceW]
   __shared__ int s_idx[32];
   __shared__ float s_p[32];
   __shared__ float s_g[128], s_u[128];
@@ -121,12 +129,16 @@ gateup_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ lo
   if (q == 0 && blockIdx.y == 0 && threadIdx.x == 0) w.status[0] = 0u;
   if (warp == 0)
     route_token<PER>(logits + (size_t)t * d.E, d.E, d.k, lane, s_idx, s_p, [](int) {});
-  // x_t -> fp32 in the decoder's K order, slice b at b * kSlice
+  // x_t -> fp16 (one rounding from the exact bf16 value, as the prefill path
+  // stages it) in the decoder's K order: word v of the row holds values
+  // pi(2v), pi(2v+1) of its K group; slice b (256 values) at b * kSliceW
   constexpr int G = Fmt<FMT>::kGroup;
-  for (int v = threadIdx.x; v < d.H; v += blockDim.x) {
-    const int g = v / G, i = v - g * G;                // position i of group g holds value perm_value(i)
-    const float f = __uint_as_float((uint32_t)__ldg(x + (size_t)t * d.H + g * G + perm_value<FMT>(i)) << 16);
-    xs[(v >> 8) * kSlice + (v & 255)] = f;
+  for (int v = threadIdx.x; v < d.H / 2; v += blockDim.x) {
+    const int g = (2 * v) / G, i = 2 * v - g * G;
+    const uint16_t* xr = x + (size_t)t * d.H + g * G;
+    const float a = __uint_as_float((uint32_t)__ldg(xr + perm_value<FMT>(i)) << 16);
+    const float b = __uint_as_float((uint32_t)__ldg(xr + perm_value<FMT>(i + 1)) << 16);
+    xs2[(v >> 7) * kSliceW + (v & 127)] = __floats2half2_rn(a, b);
   }
   __syncthreads();
   if (blockIdx.y == 0 && threadIdx.x < 32 && j == 0) {
@@ -149,7 +161,7 @@ gateup_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ lo
   if (r < d.I) {
     const size_t rowbytes = (size_t)nb * d.bb;
     const uint8_t* blk = blob + ((size_t)which * d.I + r) * rowbytes + (size_t)b * d.bb;
-    s = block_dot<FMT>(blk, xs + b * kSlice);
+    s = block_dot<FMT>(blk, xs2 + b * kSliceW);
   }
   for (int o = 1; o < nb; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (b == 0) (which ? s_u : s_g)[rl] = s;
@@ -163,32 +175,50 @@ gateup_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ lo
   }
 }
 
-// Launch 2.  grid (T, ceil(H / 8)), 256 threads: warp = output column.
+// Launch 2.  grid (T, ceil(H / kDownCols)), 256 threads; dynamic shared
+// memory: k * nbI * kSliceW fp16x2 words (the token's k rows of h, rounded
+// to fp16 as on the prefill path).  Warp w computes columns
+// c0 + 4w .. c0 + 4w + 3; lane (j, block) decodes one block of row c of
+// expert idx[t, j]'s down matrix.
 template <int FMT>
 __global__ void __launch_bounds__(kThreads)
 down_combine_small_kernel(Dims d, Work w, ExpertTable tab, const float* __restrict__ h32, float* __restrict__ y) {
   pdl_wait();
+  extern __shared__ __align__(16) __half2 hs2[];    // [k][nbI][kSliceW]
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.y * 8 + warp;
-  if (c >= d.H) return;
   const int nb = d.nbI;                                // lanes per expert
+  const int rowj = nb * kSliceW;                       // words per pair row in shared memory
+  // stage the token's k rows of h (fp32, decoder K order) as fp16x2
+  const float2* hsrc = reinterpret_cast<const float2*>(h32 + (size_t)t * d.k * d.I);
+  for (int v = threadIdx.x; v < d.k * d.I / 2; v += blockDim.x) {
+    const int jj = v / (d.I / 2), u = v - jj * (d.I / 2);
+    const float2 f = hsrc[v];
+    hs2[jj * rowj + (u >> 7) * kSliceW + (u & 127)] = __floats2half2_rn(f.x, f.y);
+  }
+  __syncthreads();
   const int j = lane / nb, b = lane - j * nb;
-  float s = 0.f;
-  if (j < d.k) {
+  const bool active = j < d.k;
+  const uint8_t* down0 = nullptr;
+  if (active) {
     const int e = __ldg(w.idx + (size_t)t * d.k + j);
-    const size_t gu_bytes = (size_t)2 * d.I * d.nbH * d.bb;
-    const uint8_t* blk = tab.p[e] + gu_bytes + ((size_t)c * nb + b) * d.bb;
-    s = block_dot<FMT>(blk, h32 + ((size_t)t * d.k + j) * d.I + b * kBlockVals);
+    down0 = tab.p[e] + (size_t)2 * d.I * d.nbH * d.bb + (size_t)b * d.bb;
   }
-  for (int o = 1; o < nb; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  // y[t, c] = sum_j p_j o_j, added in selection order j = 0, 1, ...
-  float acc = 0.f;
-  for (int jj = 0; jj < d.k; ++jj) {
-    const float oj = __shfl_sync(0xffffffffu, s, jj * nb);
-    if (lane == 0) acc = fmaf(__ldg(w.pw + (size_t)t * d.k + jj), oj, acc);
+  const __half2* hj = hs2 + j * rowj + b * kSliceW;
+  for (int cc = 0; cc < kDownCols / 8; ++cc) {
+    const int c = blockIdx.y * kDownCols + warp * (kDownCols / 8) + cc;
+    if (c >= d.H) break;                               // warp-uniform
+    float s = 0.f;
+    if (active) s = block_dot<FMT>(down0 + (size_t)c * nb * d.bb, hj);
+    for (int o = 1; o < nb; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    // y[t, c] = sum_j p_j o_j, added in selection order j = 0, 1, ...
+    float acc = 0.f;
+    for (int jj = 0; jj < d.k; ++jj) {
+      const float oj = __shfl_sync(0xffffffffu, s, jj * nb);
+      if (lane == 0) acc = fmaf(__ldg(w.pw + (size_t)t * d.k + jj), oj, acc);
+    }
+    if (lane == 0) y[(size_t)t * d.H + c] = acc;
   }
-  if (lane == 0) y[(size_t)t * d.H + c] = acc;
 }
 
 }  // namespace small

@@ -27,9 +27,11 @@ from bit_routed_expert_top_b200 import api  # noqa: E402
 def _tc_default():
     api.debug_set_gemm("tc")
     api.debug_set_path("auto")
+    api.debug_set_raw_tma(True)
     yield
     api.debug_set_gemm("tc")
     api.debug_set_path("auto")
+    api.debug_set_raw_tma(True)
 
 
 def run_prefill(inp, ws=None):
@@ -310,6 +312,41 @@ def test_edge_blocks_every_output(wl):
     h, o = workspace_h_o(ws, wl, ref["pair_pos"])
     assert Hh.y_errors(h, ref["h"])[0] < 2e-3
     assert Hh.y_errors(o, ref["o"])[0] < 2e-3
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_Q2, synth.FMT_Q1])
+def test_raw_fetch_by_tma_and_by_cp_async_agree(fmt):
+    """Rows of 2,048 values: the gate/up raw blocks come by TMA (one map over
+    the experts at their fixed stride) or, switched off, by per-lane cp.async;
+    the decoded operands are the same, so y is equal bit for bit, and within
+    tolerance of the oracle."""
+    wl = synth.Workload("rawtma", 96, 2048, 256, 16, 3, fmt)
+    inp = synth.make_inputs(wl, seed=31)
+    ref = full_oracle(inp)
+    y_tma, _ = run_prefill(inp)
+    Hh.assert_y_close(y_tma, ref["y"], "raw by TMA")
+    api.debug_set_raw_tma(False)
+    y_cp, _ = run_prefill(inp)
+    np.testing.assert_array_equal(y_tma, y_cp)
+
+
+def test_expert_table_without_a_fixed_stride():
+    """Experts stored in a shuffled order (the table has no fixed stride, so
+    the raw blocks come by cp.async) give the same y as the same experts at
+    a fixed stride."""
+    wl = synth.Workload("shuf", 80, 2048, 256, 12, 2, synth.FMT_Q2)
+    inp = synth.make_inputs(wl, seed=33)
+    y_ref, _ = run_prefill(inp)
+    perm = np.random.default_rng(2).permutation(wl.E)
+    x, logits, _ = Hh.to_device(inp)
+    shuffled = torch.from_numpy(inp.blobs[perm].copy()).cuda()      # expert perm[i] at row i
+    where = np.argsort(perm)                                           # row of expert e
+    ptrs = [shuffled[int(where[e])] for e in range(wl.E)]
+    y = torch.full((wl.T, wl.H), float("nan"), dtype=torch.float32, device="cuda")
+    ws = api.alloc_workspace(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k)
+    api.rl_moe_prefill_ws(x, logits, ptrs, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws)
+    assert api.rl_moe_check_status(ws) == 0, api.rl_last_error()
+    np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
 
 
 def test_tc_matches_simt_stage_path():
