@@ -79,17 +79,18 @@ constexpr int kNtDn = kNT;       // down unit size in pairs
 constexpr int kMtDn = 2;         // 128-row slabs per down unit
 constexpr int kMT = 2;           // M tiles per unit (gate+up, or two down slabs)
 constexpr int kAccBufs = 2;      // accumulator buffers (epilogue overlap)
-constexpr int kStepVals = 64;    // K values per decode step (two sub-blocks)
-constexpr int kRingSlotCols = 2 * 32;                                   // both tiles, 64 K values
+constexpr int kStepVals = 128;   // K values per decode step (four sub-blocks, one B stage)
+constexpr int kSlotCols = 64;    // TMEM columns of one tile's step: 128 fp16 of K per lane
+constexpr int kRingSlotCols = kMT * kSlotCols;  // both tiles
 constexpr int kRingCol = kAccBufs * kMT * kNT;  // first ring column
-constexpr int kRing = (512 - kRingCol) / kRingSlotCols;                 // A step stages in TMEM
-constexpr int kSlotCols = 32;                   // 64 fp16 of K per lane
+constexpr int kRing = 2;                        // A slots in TMEM: one per decoder phase
 constexpr int kRawStages = RL_TC_RAW_STAGES;
 constexpr int kBStages = RL_TC_B_STAGES;
 constexpr int kBK = 128;                        // K values per B stage
 constexpr int kBKBlock = 64;                    // K values per 128-byte swizzled row
 constexpr int kBBlockBytes = kNT * 128;         // one K block: kNT rows x 128 bytes
 constexpr int kBStageBytes = (kBK / kBKBlock) * kBBlockBytes;
+static_assert(kBK == kStepVals, "one B stage per decode step");
 constexpr int kRows = kMT * 128;                // weight rows per unit
 constexpr int kEpiWarp0 = 2;
 constexpr int kDecWarp0 = 6;
@@ -100,7 +101,8 @@ constexpr int kWarps = kFetchWarp0 + kMT;
 constexpr int kThreads = kWarps * 32;
 constexpr int kUnitCache = 64;                  // this CTA's first work units, cached in shared memory
 constexpr int kSharedBytes = 4096;              // barriers, work-unit cache, pair tokens
-static_assert(kRingCol + kRing * kMT * kSlotCols <= 512, "TMEM columns");
+static_assert(kRingCol + kRing * kRingSlotCols <= 512, "TMEM columns");
+static_assert(kRing == RL_TC_DEC_PHASES, "each decoder phase owns one ring slot");
 static_assert(kMT == 2, "the MMA issue below is written for two M tiles");
 
 template <int FMT> struct Raw;
@@ -211,45 +213,67 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // by a whole converged warp with warp-uniform operands through one elected
 // lane (operands then live in uniform registers: issuing from a divergent
 // single lane measured ~2x slower per instruction).
-// One 64-value step for both M tiles under a single elect: MMAs k = 0..3
-// (k = 2, 3 only when `full`) of tile t read A at a + 32t + 8k and B at
-// b + 2k (the descriptor address field counts 16-byte units: 16 fp16 of K
-// are 32 bytes inside a swizzled row), accumulate into d + kNT*t (overwrite
-// on `acc` = 0), then commit to `bar` (arrives when all of them have run).
-__device__ __forceinline__ void mma_step2x(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc,
-                                           uint32_t full, uint64_t* bar) {
+// One 128-value step for both M tiles under a single elect: MMA k
+// (k = 0..7, K values 16k..16k+15; only k < nk) of tile t reads A at
+// a + 64t + 8k and B at b + 512*(k / 4) + 2*(k % 4) (the descriptor address
+// counts 16-byte units: a 64-value K block of B is kNT rows x 128 bytes,
+// 16 fp16 of K are 32 bytes inside a swizzled row), accumulates into
+// d + kNT*t (overwrites on k = 0 when `acc` = 0), then commits to `bar`
+// (arrives when all of them have run).
+__device__ __forceinline__ void mma_step128(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                            uint32_t nk, uint64_t* bar) {
   asm volatile(
-      "{\n\t.reg .pred e, p, t, h, eh;\n\t.reg .b32 rx, d1, a1, a2, a3, a4, a5, a6, a7;\n\t"
-      ".reg .b64 b1, b2, b3;\n\t"
+      "{\n\t.reg .pred e, p0, t, q1, q2, q3, q4, q5, q6, q7;\n\t.reg .b32 rx, d1;\n\t"
+      ".reg .b32 a0h, a1l, a1h, a2l, a2h, a3l, a3h, a4l, a4h, a5l, a5h, a6l, a6h, a7l, a7h;\n\t"
+      ".reg .b64 b1, b2, b3, b4, b5, b6, b7;\n\t"
       "elect.sync rx|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
       "setp.eq.b32 t, %4, %4;\n\t"
-      "setp.ne.b32 h, %5, 0;\n\t"
-      "and.pred eh, e, h;\n\t"
+      "setp.gt.and.u32 q1, %5, 1, e;\n\t"
+      "setp.gt.and.u32 q2, %5, 2, e;\n\t"
+      "setp.gt.and.u32 q3, %5, 3, e;\n\t"
+      "setp.gt.and.u32 q4, %5, 4, e;\n\t"
+      "setp.gt.and.u32 q5, %5, 5, e;\n\t"
+      "setp.gt.and.u32 q6, %5, 6, e;\n\t"
+      "setp.gt.and.u32 q7, %5, 7, e;\n\t"
       "add.u32 d1, %0, %7;\n\t"
-      "add.u32 a1, %1, 32;\n\t"
-      "add.u32 a2, %1, 8;\n\t"
-      "add.u32 a3, %1, 40;\n\t"
-      "add.u32 a4, %1, 16;\n\t"
-      "add.u32 a5, %1, 48;\n\t"
-      "add.u32 a6, %1, 24;\n\t"
-      "add.u32 a7, %1, 56;\n\t"
+      "add.u32 a0h, %1, 64;\n\t"
+      "add.u32 a1l, %1, 8;\n\t  add.u32 a1h, %1, 72;\n\t"
+      "add.u32 a2l, %1, 16;\n\t add.u32 a2h, %1, 80;\n\t"
+      "add.u32 a3l, %1, 24;\n\t add.u32 a3h, %1, 88;\n\t"
+      "add.u32 a4l, %1, 32;\n\t add.u32 a4h, %1, 96;\n\t"
+      "add.u32 a5l, %1, 40;\n\t add.u32 a5h, %1, 104;\n\t"
+      "add.u32 a6l, %1, 48;\n\t add.u32 a6h, %1, 112;\n\t"
+      "add.u32 a7l, %1, 56;\n\t add.u32 a7h, %1, 120;\n\t"
       "add.s64 b1, %2, 2;\n\t"
       "add.s64 b2, %2, 4;\n\t"
       "add.s64 b3, %2, 6;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], %2, %3, p;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b1, %3, t;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [d1], [a3], b1, %3, t;\n\t"
-      "@eh tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b2, %3, t;\n\t"
-      "@eh tcgen05.mma.cta_group::1.kind::f16 [d1], [a5], b2, %3, t;\n\t"
-      "@eh tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b3, %3, t;\n\t"
-      "@eh tcgen05.mma.cta_group::1.kind::f16 [d1], [a7], b3, %3, t;\n\t"
+      "add.s64 b4, %2, 512;\n\t"
+      "add.s64 b5, %2, 514;\n\t"
+      "add.s64 b6, %2, 516;\n\t"
+      "add.s64 b7, %2, 518;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [d1], [a0h], %2, %3, p0;\n\t"
+      "@q1 tcgen05.mma.cta_group::1.kind::f16 [%0], [a1l], b1, %3, t;\n\t"
+      "@q1 tcgen05.mma.cta_group::1.kind::f16 [d1], [a1h], b1, %3, t;\n\t"
+      "@q2 tcgen05.mma.cta_group::1.kind::f16 [%0], [a2l], b2, %3, t;\n\t"
+      "@q2 tcgen05.mma.cta_group::1.kind::f16 [d1], [a2h], b2, %3, t;\n\t"
+      "@q3 tcgen05.mma.cta_group::1.kind::f16 [%0], [a3l], b3, %3, t;\n\t"
+      "@q3 tcgen05.mma.cta_group::1.kind::f16 [d1], [a3h], b3, %3, t;\n\t"
+      "@q4 tcgen05.mma.cta_group::1.kind::f16 [%0], [a4l], b4, %3, t;\n\t"
+      "@q4 tcgen05.mma.cta_group::1.kind::f16 [d1], [a4h], b4, %3, t;\n\t"
+      "@q5 tcgen05.mma.cta_group::1.kind::f16 [%0], [a5l], b5, %3, t;\n\t"
+      "@q5 tcgen05.mma.cta_group::1.kind::f16 [d1], [a5h], b5, %3, t;\n\t"
+      "@q6 tcgen05.mma.cta_group::1.kind::f16 [%0], [a6l], b6, %3, t;\n\t"
+      "@q6 tcgen05.mma.cta_group::1.kind::f16 [d1], [a6h], b6, %3, t;\n\t"
+      "@q7 tcgen05.mma.cta_group::1.kind::f16 [%0], [a7l], b7, %3, t;\n\t"
+      "@q7 tcgen05.mma.cta_group::1.kind::f16 [d1], [a7h], b7, %3, t;\n\t"
       "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}" ::"r"(d),
-      "r"(a), "l"(b), "r"(idesc), "r"(acc), "r"(full), "r"(smem_addr(bar)), "n"(kNT)
+      "r"(a), "l"(b), "r"(idesc), "r"(acc), "r"(nk), "r"(smem_addr(bar)), "n"(kNT)
       : "memory");
 }
-static_assert(kSlotCols == 32, "mma_step2x addresses tile 1's A at +32 columns");
+static_assert(kSlotCols == 64, "mma_step128 addresses tile 1's A at +64 columns");
+static_assert(kBBlockBytes == 8192, "mma_step128 steps the B descriptor by 512 units per 64-value K block");
 
 // Arrive on bar when every MMA issued so far by this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -541,7 +565,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
   const int lane = threadIdx.x & 31;
   const int K = GATEUP ? d.H : d.I;
   const int nsub = K / kSubVals;
-  const int nstep = (nsub + 1) / 2;
+  const int nstep = (nsub + 3) / 4;             // 128-value steps per unit
   const int nblk = GATEUP ? d.nbH : d.nbI;
   const int nbchunk = (K + kBK - 1) / kBK;
   const size_t rowbytes = (size_t)nblk * BB;
@@ -599,10 +623,8 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
   if (warp == 0) {
     // ------------------------------------------------------------ MMA ---
     // The whole warp runs this loop in lockstep; one elected lane issues.
-    // Ring slot / B stage indices and their phase bits advance incrementally;
-    // the loop body covers one B stage (two steps).
-    constexpr int kStepsPerB = kBK / kStepVals;
-    static_assert(kStepsPerB == 2, "one B stage = two decode steps");
+    // A slot (= step parity) and B stage indices and their phase bits
+    // advance incrementally; one step = one B stage = 128 K values.
     uint32_t as = 0, aph = 0, bs = 0, bph = 0;
     bool ok = true;
     const uint64_t bdesc0 = sdesc_sw128(smem_addr(b_base));
@@ -616,22 +638,14 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
         ok = wait_bar_warp(&sh->acc_empty[buf], ((ui / kAccBufs) - 1) & 1, sh, w.status, RL_TC_MMA_SLEEP_NS);
       tc_fence_after();
       const uint32_t acc0 = tmem + buf * (kMT * kNT);
-      for (int st = 0; st < nstep && ok; st += kStepsPerB) {
+      for (int st = 0; st < nstep && ok; ++st) {
         if (!wait_bar_warp(&sh->full_b[bs], bph, sh, w.status, RL_TC_MMA_SLEEP_NS)) { ok = false; break; }
         const uint64_t bd = bdesc0 + (uint64_t)((bs * kBStageBytes) >> 4);
-        // step st: K block 0 of the stage
         if (!wait_bar_warp(&sh->full_a[as], aph, sh, w.status, RL_TC_MMA_SLEEP_NS)) { ok = false; break; }
         tc_fence_after();
-        mma_step2x(acc0, a_base + as * (kMT * kSlotCols), bd, idesc, st != 0, 2 * st + 1 < nsub, &sh->empty_a[as]);
+        const uint32_t nk = 2u * (uint32_t)min(4, nsub - 4 * st);   // 16-value MMAs of this step
+        mma_step128(acc0, a_base + as * kRingSlotCols, bd, idesc, st != 0, nk, &sh->empty_a[as]);
         if (++as == kRing) { as = 0; aph ^= 1; }
-        // step st + 1: K block 1 of the stage
-        if (st + 1 < nstep) {
-          if (!wait_bar_warp(&sh->full_a[as], aph, sh, w.status, RL_TC_MMA_SLEEP_NS)) { ok = false; break; }
-          tc_fence_after();
-          mma_step2x(acc0, a_base + as * (kMT * kSlotCols), bd + (kBBlockBytes >> 4), idesc, 1u,
-                     2 * st + 3 < nsub, &sh->empty_a[as]);
-          if (++as == kRing) { as = 0; aph ^= 1; }
-        }
         mma_commit(&sh->empty_b[bs]);
         if (++bs == kBStages) { bs = 0; bph ^= 1; }
       }
@@ -721,12 +735,19 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     }
   } else if (warp < kFetchWarp0) {
     // ------------------------------------------------------ decoders -----
+    // Steps of 128 values (half a block, four sub-blocks); global step g of
+    // the CTA (counted over its units) goes to decoder phase g & 1 and TMEM
+    // ring slot g & 1, so each phase owns one slot and reuses it every
+    // other step (one lap).  Every decoder warp waits on and releases every
+    // raw stage, decoding the half of the block that falls to its phase (if
+    // that half exists), so no early release can count toward an older use
+    // of the stage.
     const int dw = warp - kDecWarp0;          // 0 .. kDecWarps-1
     const int grp = dw >> 2;                  // (tile, phase) group of four lane quarters
     const int tile = grp % kMT, phase = grp / kMT;
     const int q = warp & 3;                   // TMEM lane quarter
     const int r = q * 32 + lane;              // lane = row inside the tile
-    const uint32_t a_col = tmem + ((uint32_t)(q * 32) << 16) + kRingCol + tile * kSlotCols;
+    const uint32_t a_col = tmem + ((uint32_t)(q * 32) << 16) + kRingCol + phase * kRingSlotCols + tile * kSlotCols;
     uint8_t* const my_region0 = raw_base + raw_row_offset<FMT>(tile, r);
     // rows a multiple of 8 bytes long: a block's offset mod 8 is the same in
     // every row (blobs are 16-byte aligned), so the code loads need no selects
@@ -746,70 +767,72 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
       rowg = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, r, gu_rowbytes, rowbytes, &R);
     };
 
-    uint32_t ring_it = 0;                     // linear index of the current unit's step 0
+    uint32_t ring_it = 0;                     // global step index of the current unit's step 0
     int ui = 0, kb = 0;
     for (int c = 0; c < total_blocks && ok; ++c) {
       row_of_unit(ui);
       const int rs = c % kRawStages;
       if (!wait_bar_warp(&sh->full_raw[rs], (c / kRawStages) & 1, sh, w.status)) { ok = false; break; }
-      const uint8_t* region = my_region0 + rs * raw_stage_bytes<FMT>();
-      const int off = (int)((reinterpret_cast<uintptr_t>(rowg) + (uintptr_t)kb * BB) & 15);
-      uint32_t h0, h1;
-      load8_unaligned(region, off, h0, h1);
-      const float dd = half_bits_to_float(h0 & 0xffffu);
-      const uint32_t S = (h0 >> 16) | ((h1 & 0xffu) << 16);
-      const uint32_t flags = (h1 >> 8) & 0xffu;
-      // steps 4*kb .. 4*kb+3 of this block; this warp takes those whose
-      // linear index is its phase mod kDecPhases
-      const int m = (int)((ring_it + 4u * kb) % kDecPhases);
-      const int j0 = (phase - m + kDecPhases) % kDecPhases;
-      auto steps = [&](auto mode_tag) {
-        constexpr int MODE = decltype(mode_tag)::value;
-        for (int j = j0; j < 4; j += kDecPhases) {
-          const int st = kb * 4 + j;
-          if (2 * st >= nsub) break;
-          const int i = 2 * j;                   // first sub-block of the step inside the block
-          const uint32_t ai = ring_it + st;
-          const int as = ai % kRing;
-          // test the ring slot now; the answer is needed only after the decode
-          const bool slot_free = mbar_test_wait(smem_addr(&sh->empty_a[as]), ((ai / kRing) & 1) ^ 1);
-          // rows past the matrix decode stale stage bytes: their accumulator
-          // rows (TMEM lanes) are never read by the epilogue
+      const int hf = (int)((ring_it ^ (uint32_t)phase) & 1u);   // this phase's half of the block
+      const int st = 2 * kb + hf;                                // unit step
+      if (4 * st < nsub) {
+        const uint32_t ai = ring_it + (uint32_t)st;              // global step: ai & 1 == phase
+        // test the slot now (its previous use must have been consumed by the
+        // MMAs); the answer is needed only after the first half's decode
+        const uint32_t par = ((ai >> 1) & 1u) ^ 1u;
+        const bool slot_free = mbar_test_wait(smem_addr(&sh->empty_a[phase]), par);
+        const uint8_t* region = my_region0 + rs * raw_stage_bytes<FMT>();
+        const int off = (int)((reinterpret_cast<uintptr_t>(rowg) + (uintptr_t)kb * BB) & 15);
+        uint32_t h0, h1;
+        load8_unaligned(region, off, h0, h1);
+        const float dd = half_bits_to_float(h0 & 0xffffu);
+        const uint32_t S = (h0 >> 16) | ((h1 & 0xffu) << 16);
+        const uint32_t flags = (h1 >> 8) & 0xffu;
+        const int i0 = 4 * hf;                // first sub-block of the step inside the block
+        // rows past the matrix decode stale stage bytes: their accumulator
+        // rows (TMEM lanes) are never read by the epilogue
+        auto halves = [&](auto mode_tag) {
+          constexpr int MODE = decltype(mode_tag)::value;
           uint32_t words[32];
-          uint32_t lo0, hi0, lo1, hi1;
-          make_lut<FMT>(dd, S, flags, i, lo0, hi0);
-          make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
-          if constexpr (FMT == RL_FMT_Q2) {
-            uint32_t cw[4];
-            load_codes<FMT, MODE>(region, off + 5 + 8 * i, cw);
-            decode_word<FMT>(cw[0], lo0, hi0, words);
-            decode_word<FMT>(cw[1], lo0, hi0, words + 8);
-            decode_word<FMT>(cw[2], lo1, hi1, words + 16);
-            decode_word<FMT>(cw[3], lo1, hi1, words + 24);
-          } else {
-            uint32_t cw[2];
-            load_codes<FMT, MODE>(region, off + 6 + 4 * i, cw);
-            decode_word<FMT>(cw[0], lo0, hi0, words);
-            decode_word<FMT>(cw[1], lo1, hi1, words + 16);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int i = i0 + 2 * hh;        // first sub-block of this half
+            uint32_t lo0, hi0, lo1, hi1;
+            make_lut<FMT>(dd, S, flags, i, lo0, hi0);
+            make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
+            if constexpr (FMT == RL_FMT_Q2) {
+              uint32_t cw[4];
+              load_codes<FMT, MODE>(region, off + 5 + 8 * i, cw);
+              decode_word<FMT>(cw[0], lo0, hi0, words);
+              decode_word<FMT>(cw[1], lo0, hi0, words + 8);
+              decode_word<FMT>(cw[2], lo1, hi1, words + 16);
+              decode_word<FMT>(cw[3], lo1, hi1, words + 24);
+            } else {
+              uint32_t cw[2];
+              load_codes<FMT, MODE>(region, off + 6 + 4 * i, cw);
+              decode_word<FMT>(cw[0], lo0, hi0, words);
+              decode_word<FMT>(cw[1], lo1, hi1, words + 16);
+            }
+            if (hh == 0) {
+              if (!__all_sync(0xffffffffu, slot_free) &&
+                  !wait_bar_warp(&sh->empty_a[phase], par, sh, w.status)) { ok = false; return; }
+              tc_fence_after();
+            }
+            tmem_st32(a_col + 32 * hh, words);
           }
-          if (!__all_sync(0xffffffffu, slot_free) &&
-              !wait_bar_warp(&sh->empty_a[as], ((ai / kRing) & 1) ^ 1, sh, w.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t dst = a_col + as * (kMT * kSlotCols);
-          tmem_st32(dst, words);
           // hand the slot to the MMA warp once the stores have landed
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          mbar_arrive_if(&sh->full_a[as], lane == 0);
-        }
-      };
-      // the code bytes of every step of this block start at the same offset
-      // mod 8 (8i and 4i*2 are multiples of 8): one warp-uniform choice
-      const int ocode = __shfl_sync(0xffffffffu, off + Fmt<FMT>::kCodeOff, 0) & 7;
-      if (!uniform8) steps(std::integral_constant<int, 0>{});
-      else if (ocode < 4) steps(std::integral_constant<int, 1>{});
-      else steps(std::integral_constant<int, 2>{});
+          mbar_arrive_if(&sh->full_a[phase], lane == 0);
+        };
+        // every step's code bytes start at the same offset mod 8 (8i is a
+        // multiple of 8): one warp-uniform choice
+        const int ocode = __shfl_sync(0xffffffffu, off + Fmt<FMT>::kCodeOff, 0) & 7;
+        if (!uniform8) halves(std::integral_constant<int, 0>{});
+        else if (ocode < 4) halves(std::integral_constant<int, 1>{});
+        else halves(std::integral_constant<int, 2>{});
+      }
       __syncwarp();
       mbar_arrive_if(&sh->empty_raw[rs], lane == 0);
       if (++kb == nblk) {

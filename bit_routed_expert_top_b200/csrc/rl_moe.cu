@@ -292,37 +292,34 @@ bool small_path_fits(const rl::Dims& d, const Layout& L) {
   return L.h16 + (size_t)d.P * d.I * 4 <= L.total;
 }
 
-template <int FMT, int PER>
-cudaError_t launch_gateup_small(const void* x, const float* logits, const rl::Dims& d, const rl::Work& w,
-                                const rl::ExpertTable& tab, float* h32, cudaStream_t s) {
-  const int rows_c = 4 * (32 / d.nbH);
-  const size_t smem = (size_t)d.nbH * rl::small::kSliceW * sizeof(__half2);
-  rl::small::gateup_small_kernel<FMT, PER><<<dim3(d.P, (d.I + rows_c - 1) / rows_c), rl::small::kThreads, smem, s>>>(
-      static_cast<const uint16_t*>(x), logits, d, w, tab, h32);
-  return cudaGetLastError();
-}
-
 template <int FMT>
 int launch_small(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
                  const rl::Work& w, float* h32, float* y, cudaStream_t s) {
   const bool prof = g_prof.load(std::memory_order_relaxed);
+  const bool pdl = !prof;
   mark(0, s);
+  const int per = (d.E + 31) / 32;
+  const dim3 rg((d.T + 7) / 8), rb(rl::small::kThreads);
+  if (per <= 1) rl::small::route_small_kernel<1><<<rg, rb, 0, s>>>(logits, d, w);
+  else if (per <= 2) rl::small::route_small_kernel<2><<<rg, rb, 0, s>>>(logits, d, w);
+  else if (per <= 4) rl::small::route_small_kernel<4><<<rg, rb, 0, s>>>(logits, d, w);
+  else if (per <= 8) rl::small::route_small_kernel<8><<<rg, rb, 0, s>>>(logits, d, w);
+  else if (per <= 16) rl::small::route_small_kernel<16><<<rg, rb, 0, s>>>(logits, d, w);
+  else rl::small::route_small_kernel<32><<<rg, rb, 0, s>>>(logits, d, w);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "route_small_kernel launch");
   mark(1, s);
   mark(2, s);
-  const int per = (d.E + 31) / 32;
-  cudaError_t e;
-  if (per <= 1) e = launch_gateup_small<FMT, 1>(x, logits, d, w, tab, h32, s);
-  else if (per <= 2) e = launch_gateup_small<FMT, 2>(x, logits, d, w, tab, h32, s);
-  else if (per <= 4) e = launch_gateup_small<FMT, 4>(x, logits, d, w, tab, h32, s);
-  else if (per <= 8) e = launch_gateup_small<FMT, 8>(x, logits, d, w, tab, h32, s);
-  else if (per <= 16) e = launch_gateup_small<FMT, 16>(x, logits, d, w, tab, h32, s);
-  else e = launch_gateup_small<FMT, 32>(x, logits, d, w, tab, h32, s);
+  const int rows_c = 4 * (32 / d.nbH);
+  const size_t smem = (size_t)d.nbH * rl::small::kSliceW * sizeof(__half2);
+  e = rl::launch_k(rl::small::gateup_small_kernel<FMT>, dim3(d.P, (d.I + rows_c - 1) / rows_c),
+                   dim3(rl::small::kThreads), smem, s, pdl, static_cast<const uint16_t*>(x), d, w, tab, h32);
   if (e != cudaSuccess) return cuda_fail(e, "gateup_small_kernel launch");
   mark(3, s);
   const size_t smem2 = (size_t)d.k * d.nbI * rl::small::kSliceW * sizeof(__half2);
   e = rl::launch_k(rl::small::down_combine_small_kernel<FMT>,
                    dim3(d.T, (d.H + rl::small::kDownCols - 1) / rl::small::kDownCols), dim3(rl::small::kThreads),
-                   smem2, s, !prof, d, w, tab, static_cast<const float*>(h32), y);
+                   smem2, s, pdl, d, w, tab, static_cast<const float*>(h32), y);
   if (e != cudaSuccess) return cuda_fail(e, "down_combine_small_kernel launch");
   mark(4, s);
   mark(5, s);

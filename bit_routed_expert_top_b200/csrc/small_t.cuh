@@ -1,5 +1,5 @@
 // small_t.cuh - the decode regime: chunks of at most kMaxPairs token/expert
-// pairs (a 1- or 2-token decode or verify step) in two launches.
+// pairs (a 1- or 2-token decode or verify step) in three short launches.
 //
 // "Red Lite dev75 - --kv f16, faster prompt ingestion", section 3 (Decode):
 // for single tokens the pages run gate/up as matrix-vector rows with a few
@@ -22,8 +22,8 @@
 //             projection's decoder).  The CTAs of chunk 0 also write idx and p.
 //   launch 2  down_combine_small_kernel, grid (token, 32-column chunk): the
 //             CTA stages the token's k rows of h in shared memory (fp16, as
-//             the prefill path rounds h); warp = 4 output columns in turn,
-//             lane (j, block) decodes one block of row c of expert idx[t,j]'s
+//             the prefill path rounds h); warp = one output column, lane
+//             (j, block) decodes one block of row c of expert idx[t,j]'s
 //             down matrix and dots it with h_{t,j}; the nbI lanes of a j add
 //             up, and lane 0 adds p_j * o_j over j = 0..k-1 in selection
 //             order into y[t, c].
@@ -44,7 +44,7 @@ namespace small {
 constexpr int kMaxPairs = 64;     // chunks up to this many pairs take this path
 constexpr int kThreads = 256;     // 8 warps
 constexpr int kSliceW = kBlockVals / 2 + 4;   // fp16x2 words per 256-value activation slice (+4: bank spread)
-constexpr int kDownCols = 32;     // output columns per CTA of launch 2 (4 per warp)
+constexpr int kDownCols = 8;      // output columns per CTA of the down launch (one per warp)
 
 // 32 bits starting at byte address p (any alignment) of global memory.  Both
 // aligned words read hold at least one byte of the block (it is >= 38 bytes
@@ -113,22 +113,30 @@ __device__ __forceinline__ float block_dot(const uint8_t* blk, const __half2* xs
   return total;
 }
 
-// Launch 1.  grid (P, ceil(I / (4 * 32 / nbH))), 256 threads; PER as in
-// route_kernel; dynamic shared memory: nbH * kSliceW fp16x2 words (x_t).
-template <int FMT, int PER>
+// Launch 1.  Routing of the chunk's tokens, one warp per token (the same
+// exact top-k as the prefill path); grid ceil(T / 8), 256 threads.
+template <int PER>
+__global__ void __launch_bounds__(kThreads) route_small_kernel(const float* __restrict__ logits, Dims d, Work w) {
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + warp;
+  if (blockIdx.x == 0 && threadIdx.x == 0) w.status[0] = 0u;
+  if (t < d.T)
+    route_token<PER>(logits + (size_t)t * d.E, d.E, d.k, lane, w.idx + (size_t)t * d.k, w.pw + (size_t)t * d.k,
+                     [](int) {});
+}
+
+// Launch 2.  grid (P, ceil(I / (4 * 32 / nbH))), 256 threads; dynamic
+// shared memory: nbH * kSliceW fp16x2 words (x_t).  x_t is staged while the
+// routing launch finishes; then the pair's expert is read from idx.
+template <int FMT>
 __global__ void __launch_bounds__(kThreads)
-gateup_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ logits, Dims d, Work w,
-                    ExpertTable tab, float* __restrict__ h32) {
+gateup_small_kernel(const uint16_t* __restrict__ x, Dims d, Work w, ExpertTable tab, float* __restrict__ h32) {
   pdl_trigger();
   extern __shared__ __align__(16) __half2 xs2[];    // [nbH][kSliceW]
-  __shared__ int s_idx[32];
-  __shared__ float s_p[32];
   __shared__ float s_g[128], s_u[128];
-  const int q = blockIdx.x, t = q / d.k, j = q - t * d.k;
+  const int q = blockIdx.x, t = q / d.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (q == 0 && blockIdx.y == 0 && threadIdx.x == 0) w.status[0] = 0u;
-  if (warp == 0)
-    route_token<PER>(logits + (size_t)t * d.E, d.E, d.k, lane, s_idx, s_p, [](int) {});
   // x_t -> fp16 (one rounding from the exact bf16 value, as the prefill path
   // stages it) in the decoder's K order: word v of the row holds values
   // pi(2v), pi(2v+1) of its K group; slice b (256 values) at b * kSliceW
@@ -140,15 +148,9 @@ gateup_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ lo
     const float b = __uint_as_float((uint32_t)__ldg(xr + perm_value<FMT>(i + 1)) << 16);
     xs2[(v >> 7) * kSliceW + (v & 127)] = __floats2half2_rn(a, b);
   }
+  pdl_wait();                                          // the routing launch has finished
+  const int e = w.idx[q];
   __syncthreads();
-  if (blockIdx.y == 0 && threadIdx.x < 32 && j == 0) {
-    // one CTA per token publishes the token's routing (for launch 2)
-    for (int jj = threadIdx.x; jj < d.k; jj += 32) {
-      w.idx[(size_t)t * d.k + jj] = s_idx[jj];
-      w.pw[(size_t)t * d.k + jj] = s_p[jj];
-    }
-  }
-  const int e = s_idx[j];
   const uint8_t* blob = tab.p[e];
   const int nb = d.nbH;                                // lanes per row
   const int rows_w = 32 / nb;                          // rows per warp
@@ -175,11 +177,10 @@ gateup_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ lo
   }
 }
 
-// Launch 2.  grid (T, ceil(H / kDownCols)), 256 threads; dynamic shared
+// Launch 3.  grid (T, ceil(H / kDownCols)), 256 threads; dynamic shared
 // memory: k * nbI * kSliceW fp16x2 words (the token's k rows of h, rounded
-// to fp16 as on the prefill path).  Warp w computes columns
-// c0 + 4w .. c0 + 4w + 3; lane (j, block) decodes one block of row c of
-// expert idx[t, j]'s down matrix.
+// to fp16 as on the prefill path).  Warp w computes column c0 + w; lane
+// (j, block) decodes one block of row c of expert idx[t, j]'s down matrix.
 template <int FMT>
 __global__ void __launch_bounds__(kThreads)
 down_combine_small_kernel(Dims d, Work w, ExpertTable tab, const float* __restrict__ h32, float* __restrict__ y) {
