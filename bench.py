@@ -352,6 +352,36 @@ def per_workload_figures(args, dev, flush, headline):
     return out
 
 
+def router_gemm_figure(args, dev, flush, wl):
+    """The router projection (x [T, H] times W_r [E, H] transposed, bf16 in,
+    fp32 out) at the workload's shape: median ms over the timed steps (L2
+    flushed before each), TFLOP/s and the fraction of the bf16 peak."""
+    import torch
+    from bit_routed_expert_top_b200 import api
+
+    peaks, src = load_peaks()
+    rng = np.random.default_rng(5)
+    x = torch.from_numpy(synth.f32_to_bf16_bits(rng.standard_normal((wl.T, wl.H), dtype=np.float32))
+                         .view(np.int16).copy()).to(dev)
+    w = torch.from_numpy(synth.router_weights(wl.E, wl.H, seed=6).view(np.int16).copy()).to(dev)
+    logits = torch.empty((wl.T, wl.E), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.warmup):
+        flush.fill_(float(i))
+        api.rl_moe_router_logits(x, w, wl.T, wl.H, wl.E, logits)
+    for i, (a, b) in enumerate(ev):
+        flush.fill_(float(i))
+        a.record(stream)
+        api.rl_moe_router_logits(x, w, wl.T, wl.H, wl.E, logits)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    tf = 2.0 * wl.T * wl.H * wl.E / (ms * 1e-3) / 1e12
+    return {"T": wl.T, "H": wl.H, "E": wl.E, "ms_median": ms, "tflops": tf, "peak": peaks["bf16_tflops"],
+            "frac": tf / peaks["bf16_tflops"], "peak_source": f"{src} bf16 dense, burst"}
+
+
 def bench_ours(args, wl, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -504,8 +534,10 @@ def bench_ours(args, wl, world, rank, local):
             raise SystemExit(f"device status 0x{bits:x} on rank {rank}: {api.rl_last_error()}")
         del graph
     per_wl = None
+    router = None
     if world == 1 and not args.no_per_workload:
         per_wl = per_workload_figures(args, dev, flush, wl.name)
+        router = router_gemm_figure(args, dev, flush, wl)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -563,6 +595,8 @@ def bench_ours(args, wl, world, rank, local):
                                           "step (inputs resident, L2 flushed outside the graph)"}
     if per_wl is not None:
         line["per_workload"] = per_wl
+    if router is not None:
+        line["router_gemm"] = router
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)

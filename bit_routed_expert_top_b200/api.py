@@ -44,6 +44,9 @@ SIGNATURES = {
     "rl_moe_cache_slot_of": (_i, [_vp, _i, ctypes.POINTER(_i)]),
     "rl_moe_cache_stats": (_i, [_vp, ctypes.POINTER(ctypes.c_longlong)]),
     "rl_moe_verify_bounded": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp, _sz, _vp, _vp]),
+    "rl_moe_router_logits": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
+    "rl_moe_router_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "rl_moe_prefill_router_ws": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
 }
 RL_CACHE_HOST_POOL = 0x1
 # Not in the public header: selects the CUDA-core decode-GEMMs for stage-by-
@@ -287,6 +290,34 @@ def rl_moe_verify_bounded(cache, x, router_logits, T, k, y, workspace, stream=No
     _check(load().rl_moe_verify_bounded(cache.handle, _ptr(x), _ptr(router_logits), T, k, _ptr(y), _ptr(workspace),
                                         nbytes, idx.ctypes.data, _stream(stream)))
     return idx
+
+
+def rl_moe_router_logits(x, w_router, T, H, E, logits, stream=None):
+    """logits [T, E] fp32 = x [T, H] bf16 times w_router [E, H] bf16, transposed."""
+    _check_buf(x, "x", _X_DTYPES, T * H)
+    _check_buf(w_router, "w_router", _X_DTYPES, E * H)
+    _check_buf(logits, "logits", (torch.float32,), T * E)
+    _need_cuda(x, w_router, logits)
+    _check(load().rl_moe_router_logits(_ptr(x), _ptr(w_router), T, H, E, _ptr(logits), _stream(stream)))
+
+
+def rl_moe_router_workspace_bytes(fmt, T, H, I, E, k) -> int:
+    n = load().rl_moe_router_workspace_bytes(fmt, T, H, I, E, k)
+    if n == 0:
+        raise RlMoeError(-1, load().rl_last_error().decode(errors="replace"))
+    return n
+
+
+def rl_moe_prefill_router_ws(x, w_router, expert_blobs, fmt, T, H, I, E, k, y, workspace, stream=None):
+    _check_buf(x, "x", _X_DTYPES, T * H)
+    _check_buf(w_router, "w_router", _X_DTYPES, E * H)
+    _check_buf(y, "y", (torch.float32,), T * H)
+    _check_buf(workspace, "workspace", (), 0)
+    _need_cuda(x, w_router, y, workspace)
+    table = expert_blobs if isinstance(expert_blobs, ctypes.Array) else expert_table(expert_blobs, E)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().rl_moe_prefill_router_ws(_ptr(x), _ptr(w_router), ctypes.cast(table, ctypes.c_void_p), fmt, T, H,
+                                           I, E, k, _ptr(y), _ptr(workspace), nbytes, _stream(stream)))
 
 
 def rl_moe_check_status(workspace, stream=None) -> int:

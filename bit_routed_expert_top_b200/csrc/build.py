@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 OUT = os.path.join(PKG, "librl_moe.so")
 SOURCES = ["rl_moe.cu", "expert_cache.cu"]
-HEADERS = ["common.cuh", "route_group.cuh", "gemm_simt.cuh", "gemm_tc.cuh", "small_t.cuh"]
+HEADERS = ["common.cuh", "route_group.cuh", "gemm_simt.cuh", "gemm_tc.cuh", "small_t.cuh", "router_gemm.cuh"]
 
 
 def nvcc():

@@ -93,6 +93,7 @@ struct Dims {
   long long expert_stride;  // bytes between consecutive experts' blobs when raw_tma
   long long wait_cycles;  // limit of every bounded device wait, in SM clock cycles
   int debug_fault;        // RL_DEBUG_* bits (0 on every normal call)
+  int keep_status;        // 1: the routing launch leaves the status word (an earlier launch of the call reset it)
 };
 
 // Debug switches of the decode-GEMMs (set by rl_moe_debug_set_fault, never on

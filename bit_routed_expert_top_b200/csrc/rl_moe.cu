@@ -16,6 +16,7 @@
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "route_group.cuh"
+#include "router_gemm.cuh"
 #include "small_t.cuh"
 
 namespace {
@@ -136,6 +137,7 @@ int plan(int fmt, int T, int H, int I, int E, int k, rl::Dims* d, Layout* L) {
   d->max_units_dn = d->groups_dn * (E + (d->P + kNtDown - 1) / kNtDown);
   d->raw_tma = 0;
   d->expert_stride = 0;
+  d->keep_status = 0;
   d->wait_cycles = g_wait_cycles.load(std::memory_order_relaxed);
   d->debug_fault = g_fault.load(std::memory_order_relaxed);
   size_t o = 0;
@@ -228,6 +230,45 @@ int make_act_map(CUtensorMap* map, const void* base, int K, long long rows, int 
                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(RL_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
   return RL_OK;
+}
+
+// bf16 [rows][K] row-major, 128-byte swizzled boxes of 64 x 128 (router GEMM operands).
+int make_bf16_map(CUtensorMap* map, const void* base, int K, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(RL_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {64u, 128u};
+  const cuuint32_t es[2] = {1u, 1u};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RL_ERR_CUDA, "cuTensorMapEncodeTiled (bf16) failed (CUresult %d)", (int)r);
+  return RL_OK;
+}
+
+// logits = x W_r^T (router_gemm.cuh).  status may be null.
+int launch_router(const void* x, const void* wr, int T, int H, int E, float* logits, unsigned* status,
+                  cudaStream_t s) {
+  static std::atomic<unsigned long long> configured{0};
+  const int dev = current_device();
+  const unsigned long long bit = dev >= 0 && dev < kMaxDevices ? 1ull << dev : 0ull;
+  if (!(configured.load(std::memory_order_acquire) & bit)) {
+    const cudaError_t e = cudaFuncSetAttribute(rl::router::router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               rl::router::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(router_gemm_kernel)");
+    configured.fetch_or(bit, std::memory_order_release);
+  }
+  alignas(64) CUtensorMap xmap, wmap;
+  int rc = make_bf16_map(&xmap, x, H, T);
+  if (rc != RL_OK) return rc;
+  rc = make_bf16_map(&wmap, wr, H, E);
+  if (rc != RL_OK) return rc;
+  const dim3 grid((T + rl::router::kTM - 1) / rl::router::kTM, (E + rl::router::kTN - 1) / rl::router::kTN);
+  const cudaError_t e = rl::launch_k(rl::router::router_gemm_kernel, grid, dim3(rl::router::kThreads),
+                                     rl::router::kSmemBytes, s, false, xmap, wmap, T, H, E, logits, status,
+                                     (long long)g_wait_cycles.load(std::memory_order_relaxed));
+  return e == cudaSuccess ? RL_OK : cuda_fail(e, "router_gemm_kernel launch");
 }
 
 // The gate/up raw blocks of every expert as one 3-D uint8 tensor: x = byte
@@ -455,6 +496,58 @@ int rl_moe_prefill_ws(const void* x, const float* router_logits, const void* con
   }
   return fmt == RL_FMT_Q2 ? launch_all<RL_FMT_Q2>(x, router_logits, tab, d, w, y, s)
                           : launch_all<RL_FMT_Q1>(x, router_logits, tab, d, w, y, s);
+}
+
+int rl_moe_router_logits(const void* x, const void* w_router, int T, int H, int E, float* logits, void* stream) {
+  if (T < 0 || H <= 0 || E < 1 || H % 32 || H > RL_MAX_DIM || E > RL_MAX_EXPERTS)
+    return fail(RL_ERR_INVALID_ARG, "T=%d, H=%d, E=%d outside the limits", T, H, E);
+  if (T == 0) return RL_OK;
+  if (!x || !w_router || !logits) return fail(RL_ERR_INVALID_ARG, "NULL x, w_router or logits");
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(w_router) % 16 ||
+      reinterpret_cast<uintptr_t>(logits) % 16)
+    return fail(RL_ERR_INVALID_ARG, "x, w_router and logits must be 16-byte aligned");
+  return launch_router(x, w_router, T, H, E, logits, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+size_t rl_moe_router_workspace_bytes(int fmt, int T, int H, int I, int E, int k) {
+  const size_t n = rl_moe_workspace_bytes(fmt, T, H, I, E, k);
+  return n ? n + align_up((size_t)T * E * 4, 256) : 0;
+}
+
+int rl_moe_prefill_router_ws(const void* x, const void* w_router, const void* const* expert_blobs, int fmt, int T,
+                             int H, int I, int E, int k, float* y, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  rl::Dims d;
+  Layout L;
+  int rc = plan(fmt, T, H, I, E, k, &d, &L);
+  if (rc != RL_OK) return rc;
+  if (T == 0) return RL_OK;
+  if (!x || !w_router || !y || !workspace)
+    return fail(RL_ERR_INVALID_ARG, "NULL x, w_router, y or workspace");
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(w_router) % 16 ||
+      reinterpret_cast<uintptr_t>(y) % 16 || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(RL_ERR_INVALID_ARG, "x, w_router and y must be 16-byte aligned, workspace 256-byte aligned");
+  const size_t need = L.total + align_up((size_t)T * E * 4, 256);
+  if (ws_bytes < need) return fail(RL_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, need);
+  static thread_local rl::ExpertTable tab;
+  rc = fill_table(expert_blobs, E, &tab);
+  if (rc != RL_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const rl::Work w = carve(workspace, L);
+  float* logits = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.total);
+  // the call's status word is cleared here, so the routing launch keeps it
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  rc = launch_router(x, w_router, T, H, E, logits, w.status, s);
+  if (rc != RL_OK) return rc;
+  d.keep_status = 1;
+  if (small_path_fits(d, L)) {
+    float* h32 = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.h16);
+    return fmt == RL_FMT_Q2 ? launch_small<RL_FMT_Q2>(x, logits, tab, d, w, h32, y, s)
+                            : launch_small<RL_FMT_Q1>(x, logits, tab, d, w, h32, y, s);
+  }
+  return fmt == RL_FMT_Q2 ? launch_all<RL_FMT_Q2>(x, logits, tab, d, w, y, s)
+                          : launch_all<RL_FMT_Q1>(x, logits, tab, d, w, y, s);
 }
 
 int rl_moe_prefill(const void* x, const float* router_logits, const void* const* expert_blobs,

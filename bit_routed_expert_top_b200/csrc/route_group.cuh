@@ -97,7 +97,7 @@ route_kernel(const float* __restrict__ logits, Dims d, Work w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
   if (blockIdx.x == 0) {
-    if (threadIdx.x == 0) w.status[0] = 0u;
+    if (threadIdx.x == 0 && !d.keep_status) w.status[0] = 0u;
     for (int i = threadIdx.x; i < kMaxGroupCtas; i += blockDim.x) w.look[i] = 0ull;
   }
   for (int e = threadIdx.x; e < d.E; e += blockDim.x) smask[e] = 0u;

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kThreads) route_small_kernel(const float* __re
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
-  if (blockIdx.x == 0 && threadIdx.x == 0) w.status[0] = 0u;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && !d.keep_status) w.status[0] = 0u;
   if (t < d.T)
     route_token<PER>(logits + (size_t)t * d.E, d.E, d.k, lane, w.idx + (size_t)t * d.k, w.pw + (size_t)t * d.k,
                      [](int) {});

@@ -152,6 +152,15 @@ def make_inputs(wl: Workload, seed: int | None = None) -> Inputs:
     return Inputs(wl, x_bits, logits, blobs, seed)
 
 
+def router_weights(E: int, H: int, seed: int) -> np.ndarray:
+    """Router weights W_r [E, H] as bf16 bit patterns: float32 N(0, 1/H)
+    rounded to bf16, so that with x ~ N(0,1) the logits are about N(0, 1)
+    like the other workloads' logits."""
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((E, H), dtype=np.float32) / np.float32(np.sqrt(H))
+    return f32_to_bf16_bits(w)
+
+
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     """Exact widening of bf16 bit patterns to float32 (a bit shift, no rounding)."""
     return (bits.astype(np.uint32) << 16).view(np.float32)

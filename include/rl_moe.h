@@ -130,6 +130,35 @@ int rl_moe_prefill_ws(const void* x, const float* router_logits,
                       int I, int E, int k, float* y, void* workspace,
                       size_t ws_bytes, void* stream);
 
+/*
+ * The router projection upstream of step 1 ("Red Lite dev72 - bounded
+ * verify, profiling", section 1: the router runs per row before the
+ * experts; "Red Lite dev75 - --kv f16, faster prompt ingestion", section 2:
+ * the dense work around the routed experts): logits[t, e] = sum_h x[t, h] *
+ * w_router[e, h], bf16 operands, fp32 sums on the tensor cores.
+ *   x        device, bf16 [T, H] row-major; w_router device, bf16 [E, H]
+ *            row-major; both 16-byte aligned.  H a multiple of 32.
+ *   logits   device, fp32 [T, E] row-major, overwritten, 16-byte aligned.
+ * The sums run in an order of the hardware's choosing, so a logit may differ
+ * from an exactly rounded one by the fp32 accumulation error (a few ulps of
+ * sum_h |x w|); near-ties between experts may then rank differently from an
+ * exact evaluation.  A wait that runs out is not reported (no workspace).
+ */
+int rl_moe_router_logits(const void* x, const void* w_router, int T, int H, int E, float* logits,
+                         void* stream);
+
+/* Workspace bytes of rl_moe_prefill_router_ws (the layer's workspace plus
+ * the [T, E] fp32 logits); 0 on a bad argument. */
+size_t rl_moe_router_workspace_bytes(int fmt, int T, int H, int I, int E, int k);
+
+/* The layer from x and the router weights: rl_moe_router_logits into the
+ * workspace, then rl_moe_prefill_ws on those logits (same arguments, with
+ * w_router in place of router_logits).  Device status as for
+ * rl_moe_prefill_ws (this call clears it at its start). */
+int rl_moe_prefill_router_ws(const void* x, const void* w_router, const void* const* expert_blobs,
+                             int fmt, int T, int H, int I, int E, int k, float* y, void* workspace,
+                             size_t ws_bytes, void* stream);
+
 /* Fixed size of the scratch array used by rl_moe_prefill_noalloc (16 MiB). */
 #define RL_NOALLOC_SCRATCH_BYTES (16u << 20)
 

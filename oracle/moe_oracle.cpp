@@ -278,6 +278,23 @@ int orc_moe_prefill(int fmt, const uint16_t* x_bits, const float* logits, const 
   return orc_combine(p, o_all.data(), T, k, H, y);
 }
 
+// Router logits of T tokens over E experts: out[t*E + e] = sum over h
+// (ascending) of x[t,h] * w[e,h], both bf16 widened exactly to double, the
+// products and sums in double.  The router projection that precedes the
+// routing step ("Red Lite dev72 - bounded verify, profiling", section 1:
+// router selection per row before the experts).
+int orc_router_logits(const uint16_t* x_bits, const uint16_t* w_bits, int T, int H, int E, double* out) {
+  if (T < 0 || H <= 0 || E < 1 || (T && (!x_bits || !w_bits || !out))) return -1;
+  for (int t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h)
+        acc += bf16_to_double(x_bits[(size_t)t * H + h]) * bf16_to_double(w_bits[(size_t)e * H + h]);
+      out[(size_t)t * E + e] = acc;
+    }
+  return 0;
+}
+
 // Per-pair expert outputs o (pair-id order, [T*k, H]) of the pairs that
 // belong to experts e0 <= e < e1, from the grouped lists of orc_group; rows
 // of other experts' pairs are not written.  Each expert is decoded once and

@@ -63,6 +63,7 @@ _SIGNATURES = {
     "orc_moe_prefill": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p]),
     "orc_moe_prefill_tokens": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
     "orc_expert_outputs": (_i, [_i, _p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _i, _p]),
+    "orc_router_logits": (_i, [_p, _p, _i, _i, _i, _p]),
     "orc_hardware_concurrency": (ctypes.c_uint, []),
 }
 
@@ -287,6 +288,20 @@ def moe_prefill_tokens(x_bits, logits, blobs, fmt: int, H: int, I: int, k: int, 
     """Returns (idx [n, k], p [n, k], y [n, H]) of the given tokens."""
     idx, p, y, _ = moe_prefill_tokens_timed(x_bits, logits, blobs, fmt, H, I, k, tokens)
     return idx, p, y
+
+
+def router_logits(x_bits, w_bits):
+    """logits [T, E] float64 = x [T, H] times w [E, H] transposed, both given
+    as bf16 bit patterns (exact widening, float64 products and sums)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    w_bits = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    T, H = x_bits.shape
+    E = w_bits.shape[0]
+    if w_bits.shape != (E, H):
+        raise ValueError("w must be [E, H]")
+    out = np.empty((T, E), np.float64)
+    _check(load().orc_router_logits(_ptr(x_bits), _ptr(w_bits), T, H, E, _ptr(out)), "router_logits")
+    return out
 
 
 def moe_prefill_threaded(x_bits, logits, blobs, fmt: int, H: int, I: int, k: int, threads: int = 0):

@@ -166,3 +166,21 @@ def test_bf16_widening_every_bit_pattern_against_torch():
     assert np.array_equal(np.isnan(got), nan)
     assert np.array_equal(got[~nan], want[~nan])
     assert np.array_equal(np.signbit(got[~nan]), np.signbit(want[~nan]))
+
+
+def test_router_logits_against_numpy_matmul():
+    """The oracle's router projection against numpy's matrix product of the
+    same widened bf16 operands (a library routine): equal to float64
+    rounding."""
+    rng = np.random.default_rng(12)
+    x = synth.f32_to_bf16_bits(rng.standard_normal((9, 96), dtype=np.float32))
+    w = synth.router_weights(13, 96, seed=4)
+    got = O.router_logits(x, w)
+    want = synth.bf16_bits_to_f32(x).astype(np.float64) @ synth.bf16_bits_to_f32(w).astype(np.float64).T
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    # orientation: one nonzero weight picks one input column into one expert
+    w1 = np.zeros((13, 96), np.uint16)
+    w1[5, 17] = 0x3F80                                   # 1.0 in bf16
+    l1 = O.router_logits(x, w1)
+    np.testing.assert_array_equal(l1[:, 5], synth.bf16_bits_to_f32(x[:, 17]).astype(np.float64))
+    assert np.count_nonzero(l1[:, np.arange(13) != 5]) == 0
