@@ -793,6 +793,17 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
         // rows (TMEM lanes) are never read by the epilogue
         auto halves = [&](auto mode_tag) {
           constexpr int MODE = decltype(mode_tag)::value;
+          // the code words of both halves are read before the first TMEM
+          // store (an asm statement with a memory clobber, which later
+          // shared-memory reads cannot move above)
+          constexpr int kCw = FMT == RL_FMT_Q2 ? 4 : 2;       // code words per half
+          uint32_t cw[2][kCw];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int i = i0 + 2 * hh;
+            if constexpr (FMT == RL_FMT_Q2) load_codes<FMT, MODE>(region, off + 5 + 8 * i, cw[hh]);
+            else load_codes<FMT, MODE>(region, off + 6 + 4 * i, cw[hh]);
+          }
           uint32_t words[32];
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
@@ -801,17 +812,13 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
             make_lut<FMT>(dd, S, flags, i, lo0, hi0);
             make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
             if constexpr (FMT == RL_FMT_Q2) {
-              uint32_t cw[4];
-              load_codes<FMT, MODE>(region, off + 5 + 8 * i, cw);
-              decode_word<FMT>(cw[0], lo0, hi0, words);
-              decode_word<FMT>(cw[1], lo0, hi0, words + 8);
-              decode_word<FMT>(cw[2], lo1, hi1, words + 16);
-              decode_word<FMT>(cw[3], lo1, hi1, words + 24);
+              decode_word<FMT>(cw[hh][0], lo0, hi0, words);
+              decode_word<FMT>(cw[hh][1], lo0, hi0, words + 8);
+              decode_word<FMT>(cw[hh][2], lo1, hi1, words + 16);
+              decode_word<FMT>(cw[hh][3], lo1, hi1, words + 24);
             } else {
-              uint32_t cw[2];
-              load_codes<FMT, MODE>(region, off + 6 + 4 * i, cw);
-              decode_word<FMT>(cw[0], lo0, hi0, words);
-              decode_word<FMT>(cw[1], lo1, hi1, words + 16);
+              decode_word<FMT>(cw[hh][0], lo0, hi0, words);
+              decode_word<FMT>(cw[hh][1], lo1, hi1, words + 16);
             }
             if (hh == 0) {
               if (!__all_sync(0xffffffffu, slot_free) &&

@@ -91,11 +91,13 @@ static_assert(kNtGateUp == kNtDown, "the grouping kernel derives both unit lists
 constexpr int kLaunchesPerCall = 6;
 
 // Debug switches (not in the public header): which decode-GEMM runs (0:
-// tensor cores, 1: CUDA cores), the limit of every bounded device wait, and
-// the RL_DEBUG_* fault bits.  Read once per call into its Dims.
+// tensor cores, 1: CUDA cores), which path small chunks take (0: the decode
+// regime, 1: always the prefill path), how gate/up fetches raw blocks, the
+// limit of every bounded device wait, and the RL_DEBUG_* fault bits.  Read
+// once per call into its Dims.
 std::atomic<int> g_gemm{0};
 std::atomic<int> g_path{0};
-std::atomic<int> g_raw_tma{1};  // 1: gate/up raw blocks by TMA when the expert table allows it   // 0: small chunks take the decode-regime path, 1: always the prefill path
+std::atomic<int> g_raw_tma{1};  // 1: gate/up raw blocks by TMA when the expert table allows it
 std::atomic<long long> g_wait_cycles{rl::kDefaultWaitCycles};
 std::atomic<int> g_fault{0};
 
