@@ -8,19 +8,20 @@
 // two tokens every weight is used once or twice, so the step is bound by
 // weight bytes (about 17 MB for 2 tokens x top-10 of 512 experts), and what
 // the prefill path spends on grouping, work lists and pipeline fill of the
-// persistent tensor-core kernels dominates.  Here:
+// persistent tensor-core kernels dominates.  Here, three launches chained by
+// programmatic dependent launch:
 //
-//   launch 1  gateup_small_kernel, grid (pair q = t*k + j, row chunk):
-//             every CTA routes its pair's token itself (route_token, the
-//             same exact top-k as the prefill path: no separate routing
-//             launch); it stages x_t in shared memory as fp32 in the
-//             decoder's K order, and lane (row, block) of a warp decodes one
-//             256-value block of a gate (warps 0-3) or up (warps 4-7) row and
-//             takes its dot product with x_t in fp32 (packed fp32 FMA); the
-//             nbH lanes of a row add up, and h = silu(g) * u is written in
-//             fp32 to the pair's row of h (in the K order of the down
-//             projection's decoder).  The CTAs of chunk 0 also write idx and p.
-//   launch 2  down_combine_small_kernel, grid (token, 32-column chunk): the
+//   launch 1  route_small_kernel: one warp per token, the same exact top-k
+//             and softmax as the prefill path (route_token).
+//   launch 2  gateup_small_kernel, grid (pair q = t*k + j, row chunk): the
+//             CTA stages x_t in shared memory as fp16x2 in the decoder's K
+//             order while launch 1 finishes, then reads the pair's expert;
+//             lane (row, block) of a warp decodes one 256-value block of a
+//             gate (warps 0-3) or up (warps 4-7) row and takes its dot
+//             product with x_t; the nbH lanes of a row add up, and
+//             h = silu(g) * u is written in fp32 to the pair's row of h (in
+//             the K order of the down projection's decoder).
+//   launch 3  down_combine_small_kernel, grid (token, 8-column chunk): the
 //             CTA stages the token's k rows of h in shared memory (fp16, as
 //             the prefill path rounds h); warp = one output column, lane
 //             (j, block) decodes one block of row c of expert idx[t,j]'s
@@ -30,7 +31,7 @@
 //
 // Weights, x and h are rounded to fp16 exactly as on the prefill path; the
 // products of one code word (16 values) are summed in fp16 pairs and these
-// partials in fp32.  Both kernels are plain loads and arithmetic: no waits
+// partials in fp32.  The kernels are plain loads and arithmetic: no waits
 // on other CTAs.
 #pragma once
 
