@@ -28,10 +28,12 @@ __device__ __forceinline__ unsigned route_key(float v) {
 // every byte column of the bitmap (4 per 32-bit word), so CTAs past T write
 // zero bytes and no zeroing pass is needed.
 //  - Lane l holds the logits of experts l, l+32, ... (PER per lane, PER a
-//    power of two >= E/32) and its best not-yet-taken one.  Each of the k
-//    rounds takes the warp-wide best of the lanes' bests (larger value, or
-//    equal value and lower expert index; -0.0 equals +0.0); only the winning
-//    lane rescans its own values.
+//    power of two >= E/32) and, sorted, its three best not-yet-taken ones
+//    (larger value first, equal values in ascending expert index; -0.0
+//    equals +0.0).  Each of the k rounds takes the warp-wide best of the
+//    lanes' heads (larger value, or equal value and lower expert index, by
+//    two warp reductions); the winning lane pops its head, and only a lane
+//    that has given up all three rescans its own untaken values.
 //  - z_j = expf(l_j - l_0) summed in j order, p_j = z_j / sum.
 // Top-k of one token's logits row by one warp (see route_kernel): writes
 // idx[j] and the normalised p[j] for j = 0..k-1 in selection order and calls
@@ -47,31 +49,44 @@ __device__ __forceinline__ void route_token(const float* __restrict__ row, int E
     if (e < E) v[m] = __ldg(row + e);
     else { v[m] = 0.f; taken |= 1u << m; }
   }
-  // this lane's best untaken entry
-  auto rescan = [&](float& bv, int& bi) {
-    bv = 0.f;
-    bi = -1;
+  // the lane's three best (value, expert), head first; expert -1 = none.
+  // Values are visited in ascending expert index and displace an entry only
+  // when strictly larger, so equal values keep the lower index first.
+  float b0 = 0.f, b1 = 0.f, b2 = 0.f;
+  int i0 = -1, i1 = -1, i2 = -1;
 #pragma unroll
-    for (int m = 0; m < PER; ++m) {
-      const bool free_m = !((taken >> m) & 1u);
-      // strict '>' keeps the lower index on equal values (m ascending)
-      if (free_m && (bi < 0 || v[m] > bv)) { bv = v[m]; bi = lane + 32 * m; }
+  for (int m = 0; m < PER; ++m) {
+    if ((taken >> m) & 1u) continue;
+    const float x = v[m];
+    const int e = lane + 32 * m;
+    if (i0 < 0 || x > b0) {
+      b2 = b1; i2 = i1; b1 = b0; i1 = i0; b0 = x; i0 = e;
+    } else if (i1 < 0 || x > b1) {
+      b2 = b1; i2 = i1; b1 = x; i1 = e;
+    } else if (i2 < 0 || x > b2) {
+      b2 = x; i2 = e;
     }
-  };
-  float mv;
-  int mi;
-  rescan(mv, mi);
+  }
   float l0 = 0.f, sum = 0.f, my_z = 0.f;
   for (int j = 0; j < k; ++j) {
-    // warp-wide best of the lanes' bests: the largest key, then among the
+    // warp-wide best of the lanes' heads: the largest key, then among the
     // lanes holding it the lowest expert index (two warp reductions)
-    const unsigned key = mi < 0 ? 0u : route_key(mv);
+    const unsigned key = i0 < 0 ? 0u : route_key(b0);
     const unsigned kmax = __reduce_max_sync(0xffffffffu, key);
-    const int bi = (int)__reduce_min_sync(0xffffffffu, key == kmax && mi >= 0 ? (unsigned)mi : 0xFFFFFFFFu);
-    const float bv = __shfl_sync(0xffffffffu, mv, bi & 31);
+    const int bi = (int)__reduce_min_sync(0xffffffffu, key == kmax && i0 >= 0 ? (unsigned)i0 : 0xFFFFFFFFu);
+    const float bv = __shfl_sync(0xffffffffu, b0, bi & 31);
     if ((bi & 31) == lane) {
       taken |= 1u << (bi >> 5);
-      rescan(mv, mi);
+      b0 = b1; i0 = i1; b1 = b2; i1 = i2; i2 = -1;
+      if (i0 < 0) {
+        // all three given up: the best untaken value (strict '>' keeps the
+        // lower index on equal values, m ascending)
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+          const bool free_m = !((taken >> m) & 1u);
+          if (free_m && (i0 < 0 || v[m] > b0)) { b0 = v[m]; i0 = lane + 32 * m; }
+        }
+      }
     }
     if (j == 0) l0 = bv;
     const float z = expf(bv - l0);
