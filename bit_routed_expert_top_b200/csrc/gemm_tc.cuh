@@ -758,101 +758,100 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     // rows a multiple of 8 bytes long: a block's offset mod 8 is the same in
     // every row (blobs are 16-byte aligned), so the code loads need no selects
     const bool uniform8 = (rowbytes % 8) == 0;
-    const int total_blocks = my_units * nblk;
     bool ok = true;
 
-    // Per-unit address of this thread's row (block 0): the offset of a block
-    // inside its 16-byte aligned copy follows from it.
-    int cur_ui = -1;
-    const uint8_t* rowg = nullptr;
-    auto row_of_unit = [&](int ui) {
-      if (ui == cur_ui) return;
-      cur_ui = ui;
+    // Loop state kept incrementally: raw stage rs and its phase parity rpar;
+    // the global step index ring_it of the current unit's step 0.
+    int rs = 0;
+    uint32_t rpar = 0, ring_it = 0;
+    for (int ui = 0; ui < my_units && ok; ++ui) {
+      // this thread's row (block 0) of the unit: the offset of a block inside
+      // its 16-byte aligned copy follows from it, block by block
       const int4 un = unit_at(ui);
       int R;
-      rowg = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, r, gu_rowbytes, rowbytes, &R);
-    };
-
-    uint32_t ring_it = 0;                     // global step index of the current unit's step 0
-    int ui = 0, kb = 0;
-    for (int c = 0; c < total_blocks && ok; ++c) {
-      row_of_unit(ui);
-      const int rs = c % kRawStages;
-      if (!wait_bar_warp(&sh->full_raw[rs], (c / kRawStages) & 1, sh, w.status)) { ok = false; break; }
-      const int hf = (int)((ring_it ^ (uint32_t)phase) & 1u);   // this phase's half of the block
-      const int st = 2 * kb + hf;                                // unit step
-      if (4 * st < nsub) {
-        const uint32_t ai = ring_it + (uint32_t)st;              // global step: ai & 1 == phase
-        // test the slot now (its previous use must have been consumed by the
-        // MMAs); the answer is needed only after the first half's decode
-        const uint32_t par = ((ai >> 1) & 1u) ^ 1u;
-        const bool slot_free = mbar_test_wait(smem_addr(&sh->empty_a[phase]), par);
-        const uint8_t* region = my_region0 + rs * raw_stage_bytes<FMT>();
-        const int off = (int)((reinterpret_cast<uintptr_t>(rowg) + (uintptr_t)kb * BB) & 15);
-        uint32_t h0, h1;
-        load8_unaligned(region, off, h0, h1);
-        const float dd = half_bits_to_float(h0 & 0xffffu);
-        const uint32_t S = (h0 >> 16) | ((h1 & 0xffu) << 16);
-        const uint32_t flags = (h1 >> 8) & 0xffu;
-        const int i0 = 4 * hf;                // first sub-block of the step inside the block
-        // rows past the matrix decode stale stage bytes: their accumulator
-        // rows (TMEM lanes) are never read by the epilogue
-        auto halves = [&](auto mode_tag) {
-          constexpr int MODE = decltype(mode_tag)::value;
-          // the code words of both halves are read before the first TMEM
-          // store (an asm statement with a memory clobber, which later
-          // shared-memory reads cannot move above)
-          constexpr int kCw = FMT == RL_FMT_Q2 ? 4 : 2;       // code words per half
-          uint32_t cw[2][kCw];
+      const uint8_t* rowg = tile_row<GATEUP>(d, blob_at(ui, un.x), un.y, tile, r, gu_rowbytes, rowbytes, &R);
+      int off = (int)(reinterpret_cast<uintptr_t>(rowg) & 15);
+      // the code bytes' offset mod 8 is warp-uniform when rows are a multiple
+      // of 8 bytes long (lane 0's value, advanced with the block)
+      int off_u = __shfl_sync(0xffffffffu, off, 0);
+      const int hf = (int)((ring_it ^ (uint32_t)phase) & 1u);   // this phase's half of each block
+      // A-slot parity of the unit's first step of this phase: global step
+      // ai = ring_it + hf (ai & 1 == phase); each block adds two steps, i.e.
+      // one use of the slot
+      uint32_t par = (((ring_it + (uint32_t)hf) >> 1) & 1u) ^ 1u;
+      for (int kb = 0; kb < nblk; ++kb) {
+        if (!wait_bar_warp(&sh->full_raw[rs], rpar, sh, w.status)) { ok = false; break; }
+        const int st = 2 * kb + hf;                                // unit step
+        if (4 * st < nsub) {
+          // test the slot now (its previous use must have been consumed by
+          // the MMAs); the answer is needed only after the first half's decode
+          const bool slot_free = mbar_test_wait(smem_addr(&sh->empty_a[phase]), par);
+          const uint8_t* region = my_region0 + rs * raw_stage_bytes<FMT>();
+          uint32_t h0, h1;
+          load8_unaligned(region, off, h0, h1);
+          const float dd = half_bits_to_float(h0 & 0xffffu);
+          const uint32_t S = (h0 >> 16) | ((h1 & 0xffu) << 16);
+          const uint32_t flags = (h1 >> 8) & 0xffu;
+          const int i0 = 4 * hf;                // first sub-block of the step inside the block
+          // rows past the matrix decode stale stage bytes: their accumulator
+          // rows (TMEM lanes) are never read by the epilogue
+          auto halves = [&](auto mode_tag) {
+            constexpr int MODE = decltype(mode_tag)::value;
+            // the code words of both halves are read before the first TMEM
+            // store (an asm statement with a memory clobber, which later
+            // shared-memory reads cannot move above)
+            constexpr int kCw = FMT == RL_FMT_Q2 ? 4 : 2;       // code words per half
+            uint32_t cw[2][kCw];
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int i = i0 + 2 * hh;
-            if constexpr (FMT == RL_FMT_Q2) load_codes<FMT, MODE>(region, off + 5 + 8 * i, cw[hh]);
-            else load_codes<FMT, MODE>(region, off + 6 + 4 * i, cw[hh]);
-          }
-          uint32_t words[32];
+            for (int hh = 0; hh < 2; ++hh) {
+              const int i = i0 + 2 * hh;
+              if constexpr (FMT == RL_FMT_Q2) load_codes<FMT, MODE>(region, off + 5 + 8 * i, cw[hh]);
+              else load_codes<FMT, MODE>(region, off + 6 + 4 * i, cw[hh]);
+            }
+            uint32_t words[32];
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int i = i0 + 2 * hh;        // first sub-block of this half
-            uint32_t lo0, hi0, lo1, hi1;
-            make_lut<FMT>(dd, S, flags, i, lo0, hi0);
-            make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
-            if constexpr (FMT == RL_FMT_Q2) {
-              decode_word<FMT>(cw[hh][0], lo0, hi0, words);
-              decode_word<FMT>(cw[hh][1], lo0, hi0, words + 8);
-              decode_word<FMT>(cw[hh][2], lo1, hi1, words + 16);
-              decode_word<FMT>(cw[hh][3], lo1, hi1, words + 24);
-            } else {
-              decode_word<FMT>(cw[hh][0], lo0, hi0, words);
-              decode_word<FMT>(cw[hh][1], lo1, hi1, words + 16);
+            for (int hh = 0; hh < 2; ++hh) {
+              const int i = i0 + 2 * hh;        // first sub-block of this half
+              uint32_t lo0, hi0, lo1, hi1;
+              make_lut<FMT>(dd, S, flags, i, lo0, hi0);
+              make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
+              if constexpr (FMT == RL_FMT_Q2) {
+                decode_word<FMT>(cw[hh][0], lo0, hi0, words);
+                decode_word<FMT>(cw[hh][1], lo0, hi0, words + 8);
+                decode_word<FMT>(cw[hh][2], lo1, hi1, words + 16);
+                decode_word<FMT>(cw[hh][3], lo1, hi1, words + 24);
+              } else {
+                decode_word<FMT>(cw[hh][0], lo0, hi0, words);
+                decode_word<FMT>(cw[hh][1], lo1, hi1, words + 16);
+              }
+              if (hh == 0) {
+                if (!__all_sync(0xffffffffu, slot_free) &&
+                    !wait_bar_warp(&sh->empty_a[phase], par, sh, w.status)) { ok = false; return; }
+                tc_fence_after();
+              }
+              tmem_st32(a_col + 32 * hh, words);
             }
-            if (hh == 0) {
-              if (!__all_sync(0xffffffffu, slot_free) &&
-                  !wait_bar_warp(&sh->empty_a[phase], par, sh, w.status)) { ok = false; return; }
-              tc_fence_after();
-            }
-            tmem_st32(a_col + 32 * hh, words);
-          }
-          // hand the slot to the MMA warp once the stores have landed
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          mbar_arrive_if(&sh->full_a[phase], lane == 0);
-        };
-        // every step's code bytes start at the same offset mod 8 (8i is a
-        // multiple of 8): one warp-uniform choice
-        const int ocode = __shfl_sync(0xffffffffu, off + Fmt<FMT>::kCodeOff, 0) & 7;
-        if (!uniform8) halves(std::integral_constant<int, 0>{});
-        else if (ocode < 4) halves(std::integral_constant<int, 1>{});
-        else halves(std::integral_constant<int, 2>{});
+            // hand the slot to the MMA warp once the stores have landed
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            mbar_arrive_if(&sh->full_a[phase], lane == 0);
+          };
+          // every step's code bytes start at the same offset mod 8 (8i is a
+          // multiple of 8): one warp-uniform choice
+          const int ocode = (off_u + Fmt<FMT>::kCodeOff) & 7;
+          if (!uniform8) halves(std::integral_constant<int, 0>{});
+          else if (ocode < 4) halves(std::integral_constant<int, 1>{});
+          else halves(std::integral_constant<int, 2>{});
+          par ^= 1u;
+        }
+        __syncwarp();
+        mbar_arrive_if(&sh->empty_raw[rs], lane == 0);
+        if (++rs == kRawStages) { rs = 0; rpar ^= 1u; }
+        off = (off + BB) & 15;
+        off_u = (off_u + BB) & 15;
       }
-      __syncwarp();
-      mbar_arrive_if(&sh->empty_raw[rs], lane == 0);
-      if (++kb == nblk) {
-        kb = 0;
-        ++ui;
-        ring_it += nstep;
-      }
+      ring_it += nstep;
     }
   } else {
     // ----------------------------------------------------- raw fetch -----
