@@ -378,8 +378,31 @@ def router_gemm_figure(args, dev, flush, wl):
     torch.cuda.synchronize()
     ms = statistics.median(a.elapsed_time(b) for a, b in ev)
     tf = 2.0 * wl.T * wl.H * wl.E / (ms * 1e-3) / 1e12
+    # the whole layer from x and W_r (router launch with the routing fused in
+    # its epilogue, then the expert path), against the layer from logits
+    inp = synth.make_inputs(wl)
+    blobs = torch.from_numpy(inp.blobs).to(dev)
+    table = api.expert_table(blobs, wl.E)
+    y = torch.empty((wl.T, wl.H), dtype=torch.float32, device=dev)
+    ws = torch.empty(api.rl_moe_router_workspace_bytes(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k), dtype=torch.uint8,
+                     device=dev)
+    for i in range(args.warmup):
+        flush.fill_(float(i))
+        api.rl_moe_prefill_router_ws(x, w, table, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws)
+    for i, (a, b) in enumerate(ev):
+        flush.fill_(float(i))
+        a.record(stream)
+        api.rl_moe_prefill_router_ws(x, w, table, wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws)
+        b.record(stream)
+    torch.cuda.synchronize()
+    layer_ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    if api.rl_moe_check_status(ws) != 0:
+        raise RuntimeError("router layer: device status " + api.rl_last_error())
     return {"T": wl.T, "H": wl.H, "E": wl.E, "ms_median": ms, "tflops": tf, "peak": peaks["bf16_tflops"],
-            "frac": tf / peaks["bf16_tflops"], "peak_source": f"{src} bf16 dense, burst"}
+            "frac": tf / peaks["bf16_tflops"], "peak_source": f"{src} bf16 dense, burst",
+            "layer_from_x_ms_median": layer_ms,
+            "layer_from_x_method": "rl_moe_prefill_router_ws: router GEMM with the exact top-k fused in its "
+                                   "epilogue, then grouping, decode-GEMMs and combine; median of the timed steps"}
 
 
 def bench_ours(args, wl, world, rank, local):

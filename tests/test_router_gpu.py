@@ -91,3 +91,79 @@ def test_layer_from_x_and_router_weights(wl):
     ref = O.moe_prefill(inp.x_bits, l32, Hh.oracle_blobs(inp), wl.fmt, wl.H, wl.I, wl.k, keep_intermediates=False)
     same = np.all(idx == ridx, axis=1)
     Hh.assert_y_close(y.cpu().numpy()[same], ref["y"][same], wl.name)
+
+
+def _ws_routing(ws, T, E, k):
+    """idx, p, offsets, pair list and inverse of the last call, read from the
+    workspace (its layout: a 256-byte status block, then idx [T*k], p [T*k],
+    token bitmap and per-word prefixes [E][ceil(T/32)], offsets [E+1], pair
+    list and inverse [T*k], each piece starting 256-byte aligned)."""
+    P, W = T * k, (T + 31) // 32
+    raw = ws.cpu().numpy()
+    off = [0]
+
+    def take(n):
+        at = off[0]
+        off[0] = (at + n + 255) // 256 * 256
+        return at
+
+    take(256)
+    i_idx, i_pw = take(4 * P), take(4 * P)
+    take(4 * E * W), take(4 * E * W)
+    i_off, i_list, i_pos = take(4 * (E + 1)), take(4 * P), take(4 * P)
+    get = lambda at, n, dt: raw[at:at + 4 * n].view(dt)  # noqa: E731
+    return (get(i_idx, P, np.int32).reshape(T, k), get(i_pw, P, np.float32).reshape(T, k),
+            get(i_off, E + 1, np.int32), get(i_list, P, np.int32), get(i_pos, P, np.int32))
+
+
+@pytest.mark.parametrize("T,H,I,E,k,ties", [
+    (2048, 2048, 512, 512, 10, False),     # the headline shapes
+    (100, 160, 96, 40, 8, False),          # one partial expert tile
+    (5, 2048, 512, 1024, 16, False),       # eight expert tiles, the largest fused k
+    (300, 256, 256, 300, 6, True),         # equal logits across expert tiles (duplicated router rows)
+    (64, 256, 256, 64, 17, False),         # k above the fused limit: logits, then the routing launch
+])
+def test_fused_routing_equals_routing_the_exported_logits(T, H, I, E, k, ties):
+    """The layer from x and W_r routes in the router launch's epilogue (k <=
+    16): its selections, weights, grouping and y equal, bit for bit, those of
+    rl_moe_route and rl_moe_prefill_ws on the logits rl_moe_router_logits
+    returns for the same x and W_r."""
+    wl = synth.Workload("fused", T, H, I, E, k, synth.FMT_Q2)
+    inp = synth.make_inputs(wl, seed=23)
+    w = synth.router_weights(E, H, seed=24)
+    if ties:
+        for a, b in [(3, 130), (7, 260), (129, 131), (0, 299)]:
+            w[b] = w[a]                                  # identical rows: identical logits
+    x, _, blobs = Hh.to_device(inp)
+    wd = torch.from_numpy(w.view(np.int16).copy()).cuda()
+    y = torch.full((T, H), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(api.rl_moe_router_workspace_bytes(wl.fmt, T, H, I, E, k), dtype=torch.uint8, device="cuda")
+    api.rl_moe_prefill_router_ws(x, wd, blobs, wl.fmt, T, H, I, E, k, y, ws)
+    assert api.rl_moe_check_status(ws) == 0, api.rl_last_error()
+    idx, pw, offs, plist, ppos = _ws_routing(ws, T, E, k)
+
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    api.rl_moe_router_logits(x, wd, T, H, E, logits)
+    P = T * k
+    r_idx = torch.empty(P, dtype=torch.int32, device="cuda")
+    r_w = torch.empty(P, dtype=torch.float32, device="cuda")
+    r_off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    r_list = torch.empty(P, dtype=torch.int32, device="cuda")
+    r_pos = torch.empty(P, dtype=torch.int32, device="cuda")
+    ws2 = api.alloc_workspace(wl.fmt, T, H, I, E, k)
+    api.rl_moe_route(logits, T, E, k, r_idx, r_w, r_off, r_list, r_pos, ws2)
+    np.testing.assert_array_equal(idx, r_idx.cpu().numpy().reshape(T, k))
+    np.testing.assert_array_equal(pw.view(np.uint32), r_w.cpu().numpy().reshape(T, k).view(np.uint32))
+    np.testing.assert_array_equal(offs, r_off.cpu().numpy())
+    np.testing.assert_array_equal(plist, r_list.cpu().numpy())
+    np.testing.assert_array_equal(ppos, r_pos.cpu().numpy())
+    y_ref = torch.full_like(y, float("nan"))
+    api.rl_moe_prefill_ws(x, logits, blobs, wl.fmt, T, H, I, E, k, y_ref, ws2)
+    assert torch.equal(y, y_ref)
+    if ties:
+        # the duplicated rows really tie, and the lower expert index wins
+        l = logits.cpu().numpy()
+        assert np.array_equal(l[:, 3], l[:, 130])
+        for t in range(T):
+            if 130 in idx[t]:
+                assert 3 in idx[t] and list(idx[t]).index(3) < list(idx[t]).index(130)
