@@ -389,17 +389,12 @@ __device__ __forceinline__ void make_lut(float dd, uint32_t S, uint32_t flags, i
 // values (k + 2h*P, k + (2h+1)*P) of the group, P = codes per byte, i.e.
 // position i holds value (i >> 2) + P*(i & 3).
 //
-// Per four codes: the shift as a multiply (x >> n = mulhi(x, 2^(32-n))) and
-// the selectors of bytes 0-1 as one multiply-add on the FMA pipe; the mask,
-// the selectors of bytes 2-3 (a byte permute of the first selector word)
-// and the two table permutes on the integer ALU pipe.  Measured against a
-// mad.hi for the second selector, which compiles to two instructions, this
-// takes ~11% fewer instructions per code word.
-__device__ __forceinline__ uint32_t mulhi_u32(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
+// Per four codes: the selectors of bytes 0-1 as one multiply-add on the FMA
+// pipe; the shift, the mask, the selectors of bytes 2-3 (a byte permute of
+// the first selector word) and the two table permutes on the integer ALU
+// pipe.  Measured against a mad.hi for the second selector, which compiles
+// to two instructions, this takes ~11% fewer instructions per code word; a
+// high multiply in place of the shift measured slower.
 // Byte permute with the hardware's selector semantics.  __byte_perm keeps
 // only 3 bits of each selector nibble, so with a selector that is not a
 // compile-time constant it costs a masking instruction before the permute;
@@ -416,7 +411,7 @@ __device__ __forceinline__ void decode_word(uint32_t c, uint32_t lo, uint32_t hi
   constexpr uint32_t mask = FMT == RL_FMT_Q2 ? 0x03030303u : 0x01010101u;
 #pragma unroll
   for (int k = 0; k < P; ++k) {
-    const uint32_t shifted = k == 0 ? c : mulhi_u32(c, 1u << (32 - B * k));
+    const uint32_t shifted = c >> (B * k);
     const uint32_t v = shifted & mask;
     const uint32_t sel_lo = v * 0x22u + 0x10101010u;          // selectors of bytes 0-1
     const uint32_t sel_hi = __byte_perm(sel_lo, 0u, 0x3232u);     // selectors of bytes 2-3
