@@ -378,8 +378,8 @@ def router_gemm_figure(args, dev, flush, wl):
     torch.cuda.synchronize()
     ms = statistics.median(a.elapsed_time(b) for a, b in ev)
     tf = 2.0 * wl.T * wl.H * wl.E / (ms * 1e-3) / 1e12
-    # the whole layer from x and W_r (router launch with the routing fused in
-    # its epilogue, then the expert path), against the layer from logits
+    # the whole layer from x and W_r (router launch, then the layer from its
+    # logits)
     inp = synth.make_inputs(wl)
     blobs = torch.from_numpy(inp.blobs).to(dev)
     table = api.expert_table(blobs, wl.E)
@@ -401,8 +401,8 @@ def router_gemm_figure(args, dev, flush, wl):
     return {"T": wl.T, "H": wl.H, "E": wl.E, "ms_median": ms, "tflops": tf, "peak": peaks["bf16_tflops"],
             "frac": tf / peaks["bf16_tflops"], "peak_source": f"{src} bf16 dense, burst",
             "layer_from_x_ms_median": layer_ms,
-            "layer_from_x_method": "rl_moe_prefill_router_ws: router GEMM with the exact top-k fused in its "
-                                   "epilogue, then grouping, decode-GEMMs and combine; median of the timed steps"}
+            "layer_from_x_method": "rl_moe_prefill_router_ws: router GEMM, then the layer from its logits (routing, "
+                                   "grouping, decode-GEMMs, combine); median of the timed steps"}
 
 
 def bench_ours(args, wl, world, rank, local):

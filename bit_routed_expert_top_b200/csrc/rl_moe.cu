@@ -251,7 +251,7 @@ int make_bf16_map(CUtensorMap* map, const void* base, int K, long long rows) {
 
 // logits = x W_r^T (router_gemm.cuh).  status may be null.
 int launch_router(const void* x, const void* wr, int T, int H, int E, float* logits, unsigned* status,
-                  const rl::router::RouteFuse& rf, cudaStream_t s) {
+                  cudaStream_t s) {
   static std::atomic<unsigned long long> configured{0};
   const int dev = current_device();
   const unsigned long long bit = dev >= 0 && dev < kMaxDevices ? 1ull << dev : 0ull;
@@ -269,7 +269,7 @@ int launch_router(const void* x, const void* wr, int T, int H, int E, float* log
   const dim3 grid((T + rl::router::kTM - 1) / rl::router::kTM, (E + rl::router::kTN - 1) / rl::router::kTN);
   const cudaError_t e = rl::launch_k(rl::router::router_gemm_kernel, grid, dim3(rl::router::kThreads),
                                      rl::router::kSmemBytes, s, false, xmap, wmap, T, H, E, logits, status,
-                                     (long long)g_wait_cycles.load(std::memory_order_relaxed), rf);
+                                     (long long)g_wait_cycles.load(std::memory_order_relaxed));
   return e == cudaSuccess ? RL_OK : cuda_fail(e, "router_gemm_kernel launch");
 }
 
@@ -337,21 +337,18 @@ bool small_path_fits(const rl::Dims& d, const Layout& L) {
 
 template <int FMT>
 int launch_small(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
-                 const rl::Work& w, float* h32, float* y, cudaStream_t s, bool routed = false) {
+                 const rl::Work& w, float* h32, float* y, cudaStream_t s) {
   const bool prof = g_prof.load(std::memory_order_relaxed);
   const bool pdl = !prof;
   mark(0, s);
-  // routed: the router launch has written idx and p (fused routing)
-  if (!routed) {
-    const int per = (d.E + 31) / 32;
-    const dim3 rg((d.T + 7) / 8), rb(rl::small::kThreads);
-    if (per <= 1) rl::small::route_small_kernel<1><<<rg, rb, 0, s>>>(logits, d, w);
-    else if (per <= 2) rl::small::route_small_kernel<2><<<rg, rb, 0, s>>>(logits, d, w);
-    else if (per <= 4) rl::small::route_small_kernel<4><<<rg, rb, 0, s>>>(logits, d, w);
-    else if (per <= 8) rl::small::route_small_kernel<8><<<rg, rb, 0, s>>>(logits, d, w);
-    else if (per <= 16) rl::small::route_small_kernel<16><<<rg, rb, 0, s>>>(logits, d, w);
-    else rl::small::route_small_kernel<32><<<rg, rb, 0, s>>>(logits, d, w);
-  }
+  const int per = (d.E + 31) / 32;
+  const dim3 rg((d.T + 7) / 8), rb(rl::small::kThreads);
+  if (per <= 1) rl::small::route_small_kernel<1><<<rg, rb, 0, s>>>(logits, d, w);
+  else if (per <= 2) rl::small::route_small_kernel<2><<<rg, rb, 0, s>>>(logits, d, w);
+  else if (per <= 4) rl::small::route_small_kernel<4><<<rg, rb, 0, s>>>(logits, d, w);
+  else if (per <= 8) rl::small::route_small_kernel<8><<<rg, rb, 0, s>>>(logits, d, w);
+  else if (per <= 16) rl::small::route_small_kernel<16><<<rg, rb, 0, s>>>(logits, d, w);
+  else rl::small::route_small_kernel<32><<<rg, rb, 0, s>>>(logits, d, w);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "route_small_kernel launch");
   mark(1, s);
@@ -375,15 +372,13 @@ int launch_small(const void* x, const float* logits, const rl::ExpertTable& tab,
 
 template <int FMT>
 int launch_all(const void* x, const float* logits, const rl::ExpertTable& tab, const rl::Dims& d,
-               const rl::Work& w, float* y, cudaStream_t s, bool routed = false) {
+               const rl::Work& w, float* y, cudaStream_t s) {
   const bool prof = g_prof.load(std::memory_order_relaxed);
   mark(0, s);
   // kernels after the first start while their predecessor drains
   // (programmatic dependent launch), except when stage events sit between
   const bool pdl = !prof;
-  // routed: the router launch has written idx, p and the bitmap (fused
-  // routing) and zeroed the grouping records
-  if (!routed) launch_route(logits, d, w, s);
+  launch_route(logits, d, w, s);
   mark(1, s);
   rl::launch_k(rl::group_kernel, dim3((d.E + 7) / 8), dim3(256), 0, s, pdl, d, w, 1);
   rl::launch_k(rl::place_pairs_kernel<FMT>, dim3((d.T + 7) / 8), dim3(256), 0, s, pdl,
@@ -513,26 +508,12 @@ int rl_moe_router_logits(const void* x, const void* w_router, int T, int H, int 
   if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(w_router) % 16 ||
       reinterpret_cast<uintptr_t>(logits) % 16)
     return fail(RL_ERR_INVALID_ARG, "x, w_router and logits must be 16-byte aligned");
-  rl::router::RouteFuse none{};
-  return launch_router(x, w_router, T, H, E, logits, nullptr, none, static_cast<cudaStream_t>(stream));
-}
-
-// After the layer's workspace: the router's scratch, either the logits
-// [T][E] fp32 (routing by the routing kernel) or, with the routing fused into
-// the router launch (k <= its limit), the tiles' candidate lists and the
-// per-tile tickets.
-size_t router_scratch_bytes(int T, int E, int k) {
-  const size_t logits = align_up((size_t)T * E * 4, 256);
-  if (k > rl::router::kFuseK) return logits;
-  const size_t ntn = (size_t)(E + rl::router::kTN - 1) / rl::router::kTN;
-  const size_t ntm = (size_t)(T + rl::router::kTM - 1) / rl::router::kTM;
-  const size_t fused = 2 * align_up((size_t)T * ntn * k * 4, 256) + align_up(ntm * 4, 256);
-  return logits > fused ? logits : fused;
+  return launch_router(x, w_router, T, H, E, logits, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 size_t rl_moe_router_workspace_bytes(int fmt, int T, int H, int I, int E, int k) {
   const size_t n = rl_moe_workspace_bytes(fmt, T, H, I, E, k);
-  return n ? n + router_scratch_bytes(T, E, k) : 0;
+  return n ? n + align_up((size_t)T * E * 4, 256) : 0;
 }
 
 int rl_moe_prefill_router_ws(const void* x, const void* w_router, const void* const* expert_blobs, int fmt, int T,
@@ -548,48 +529,27 @@ int rl_moe_prefill_router_ws(const void* x, const void* w_router, const void* co
   if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(w_router) % 16 ||
       reinterpret_cast<uintptr_t>(y) % 16 || reinterpret_cast<uintptr_t>(workspace) % 256)
     return fail(RL_ERR_INVALID_ARG, "x, w_router and y must be 16-byte aligned, workspace 256-byte aligned");
-  const size_t need = L.total + router_scratch_bytes(T, E, k);
+  const size_t need = L.total + align_up((size_t)T * E * 4, 256);
   if (ws_bytes < need) return fail(RL_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, need);
   static thread_local rl::ExpertTable tab;
   rc = fill_table(expert_blobs, E, &tab);
   if (rc != RL_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const rl::Work w = carve(workspace, L);
-  char* scratch = static_cast<char*>(workspace) + L.total;
-  // the call's status word is cleared here, so the later launches keep it
+  float* logits = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.total);
+  // the call's status word is cleared here, so the routing launch keeps it
   cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(unsigned), s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
-  const bool fused = k <= rl::router::kFuseK;
-  float* logits = reinterpret_cast<float*>(scratch);
-  rl::router::RouteFuse rf{};
-  if (fused) {
-    // routing in the router launch's epilogue: candidate lists and tickets
-    const int ntn = (E + rl::router::kTN - 1) / rl::router::kTN;
-    const int ntm = (T + rl::router::kTM - 1) / rl::router::kTM;
-    const size_t cbytes = align_up((size_t)T * ntn * k * 4, 256);
-    rf.k = k;
-    rf.W = d.W;
-    rf.idx = w.idx;
-    rf.pw = w.pw;
-    rf.bitmap = w.bitmap;
-    rf.look = w.look;
-    rf.cand_v = reinterpret_cast<float*>(scratch);
-    rf.cand_i = reinterpret_cast<int*>(scratch + cbytes);
-    rf.ticket = reinterpret_cast<unsigned*>(scratch + 2 * cbytes);
-    e = cudaMemsetAsync(rf.ticket, 0, (size_t)ntm * 4, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(tickets)");
-    logits = nullptr;
-  }
-  rc = launch_router(x, w_router, T, H, E, logits, w.status, rf, s);
+  rc = launch_router(x, w_router, T, H, E, logits, w.status, s);
   if (rc != RL_OK) return rc;
   d.keep_status = 1;
   if (small_path_fits(d, L)) {
     float* h32 = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.h16);
-    return fmt == RL_FMT_Q2 ? launch_small<RL_FMT_Q2>(x, logits, tab, d, w, h32, y, s, fused)
-                            : launch_small<RL_FMT_Q1>(x, logits, tab, d, w, h32, y, s, fused);
+    return fmt == RL_FMT_Q2 ? launch_small<RL_FMT_Q2>(x, logits, tab, d, w, h32, y, s)
+                            : launch_small<RL_FMT_Q1>(x, logits, tab, d, w, h32, y, s);
   }
-  return fmt == RL_FMT_Q2 ? launch_all<RL_FMT_Q2>(x, logits, tab, d, w, y, s, fused)
-                          : launch_all<RL_FMT_Q1>(x, logits, tab, d, w, y, s, fused);
+  return fmt == RL_FMT_Q2 ? launch_all<RL_FMT_Q2>(x, logits, tab, d, w, y, s)
+                          : launch_all<RL_FMT_Q1>(x, logits, tab, d, w, y, s);
 }
 
 int rl_moe_prefill(const void* x, const float* router_logits, const void* const* expert_blobs,

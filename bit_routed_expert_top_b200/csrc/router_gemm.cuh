@@ -6,12 +6,9 @@
 // where the prefill time goes around the routed experts (the dense parts of
 // the layer, the shared expert); "Red Lite dev72 - bounded verify,
 // profiling", section 1, runs the router per row before the experts.  Here
-// the router's matrix product for a whole chunk is one tcgen05 GEMM, and the
-// exact top-k of step 1 runs in its epilogue on the fp32 sums: each CTA keeps,
-// per token, the k best of its 128 experts; the last CTA of a 128-token tile
-// to finish (one ticket per tile) merges the tile's candidate lists into the
-// token's top k, the routing weights and the token bitmap, so no logits go
-// to memory and no routing launch follows.
+// the router's matrix product for a whole chunk is one tcgen05 GEMM whose
+// fp32 logits (4 MB at 2,048 tokens x 512 experts, kept in L2) feed the exact
+// top-k of step 1 in the same call.
 //
 // One CTA computes a 128-token x 128-expert tile: A = x rows (M = tokens),
 // B = W_r rows (N = experts), both K-major and brought by TMA into the
@@ -82,58 +79,11 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, long 
   return true;
 }
 
-// Routing fused into the epilogue (k <= kFuseK; k = 0: logits only).
-constexpr int kFuseK = 16;
-struct RouteFuse {
-  int k;                        // experts per token; 0: no routing in this launch
-  int W;                        // 32-token words per bitmap row
-  int* idx;                     // [T][k] selections, selection order
-  float* pw;                    // [T][k] routing weights
-  unsigned* bitmap;             // [E][W] token bitmap
-  unsigned long long* look;     // grouping records, zeroed here
-  float* cand_v;                // [T][ceil(E/128)][k] candidates of each expert tile
-  int* cand_i;
-  unsigned* ticket;             // [ceil(T/128)] tiles finished (zero before the launch; left zero)
-};
-
-// Insert (v, e) into the sorted list (bv, bi) of the k best so far: larger
-// value first, equal values in ascending expert index (-0.0 equals +0.0).
-// An entry pushed down by the insertion is re-placed by the same order, so
-// it stays ahead of an equal value of higher index.  The callers insert in
-// ascending index among equal values, so a new value equal to the k-th
-// (whose index is lower) is rejected.  cnt: entries held; thr: the k-th
-// value once the list is full.  Every array index is a compile-time
-// constant (registers, no local memory).
-__device__ __forceinline__ void topk_insert(float (&bv)[kFuseK], int (&bi)[kFuseK], int& cnt, float& thr, int k,
-                                            float v, int e) {
-  if (cnt == k && !(v > thr)) return;
-  float cv = v;
-  int ci = e;
-#pragma unroll
-  for (int p = 0; p < kFuseK; ++p) {
-    if (p < cnt) {
-      if (cv > bv[p] || (cv == bv[p] && ci < bi[p])) {
-        const float tv = bv[p]; const int ti = bi[p];
-        bv[p] = cv; bi[p] = ci; cv = tv; ci = ti;
-      }
-    } else if (p == cnt && p < k) {
-      bv[p] = cv; bi[p] = ci;
-    }
-  }
-  if (cnt < k) ++cnt;
-  if (cnt == k) {
-#pragma unroll
-    for (int p = 0; p < kFuseK; ++p)
-      if (p == k - 1) thr = bv[p];
-  }
-}
-
 // grid (ceil(T / 128), ceil(E / 128)), kThreads threads, kSmemBytes of
-// dynamic shared memory.  status may be null; logits may be null when the
-// routing is fused (rf.k > 0).
+// dynamic shared memory.  status may be null.
 __global__ void __launch_bounds__(kThreads, 1)
 router_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap, int T, int H,
-                   int E, float* __restrict__ logits, unsigned* status, long long wait_cycles, RouteFuse rf) {
+                   int E, float* __restrict__ logits, unsigned* status, long long wait_cycles) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -209,14 +159,9 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
   // ------------------------------------------------- epilogue (4 warps) ----
   __syncwarp();
   const bool have = __all_sync(0xffffffffu, wait_phase(accb, 0, wait_cycles, abort, status, true));
-  const int row = m0 + warp * 32 + lane;
-  const bool fuse = rf.k > 0;
-  float bv[kFuseK];
-  int bi[kFuseK];
-  int cnt = 0;
-  float thr = 0.f;
   if (have) {
     tc::tc_fence_after();
+    const int row = m0 + warp * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
     const bool vec = (E % 4) == 0;
 #pragma unroll 1
@@ -225,25 +170,17 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
       tc::tmem_ld16(tmem + lane_addr + c0, v);
       tc::tmem_wait_ld();
       if (row < T) {
+        float* out = logits + (size_t)row * E + n0 + c0;
         const int left = E - (n0 + c0);
-        if (fuse) {
-          // this tile's experts in ascending index
+        if (vec && left >= 16) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(out + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                                              __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+        } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (i < left) topk_insert(bv, bi, cnt, thr, rf.k, __uint_as_float(v[i]), n0 + c0 + i);
-        }
-        if (logits) {
-          float* out = logits + (size_t)row * E + n0 + c0;
-          if (vec && left >= 16) {
-#pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<float4*>(out + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                                                                __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (i < left) out[i] = __uint_as_float(v[i]);
-          }
+            if (i < left) out[i] = __uint_as_float(v[i]);
         }
       }
     }
@@ -253,72 +190,6 @@ router_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
   if (warp == 0) {
     tc::tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTN) : "memory");
-  }
-  if (!fuse) return;
-
-  // ---- fused routing: this tile's candidates, then the merge by the last
-  // CTA of the 128-token tile ----------------------------------------------
-  const int ntiles = gridDim.y;
-  if (have && row < T) {
-    const size_t base = ((size_t)row * ntiles + blockIdx.y) * rf.k;
-#pragma unroll
-    for (int p = 0; p < kFuseK; ++p) {
-      if (p < rf.k) {
-        rf.cand_v[base + p] = p < cnt ? bv[p] : 0.f;
-        rf.cand_i[base + p] = p < cnt ? bi[p] : -1;
-      }
-    }
-  }
-  __shared__ int s_last;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned old = atomicAdd(rf.ticket + blockIdx.x, 1u);
-    s_last = old == (unsigned)(ntiles - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();                                   // every tile's candidates are visible
-  __shared__ unsigned smask[RL_MAX_EXPERTS][kTM / 32];
-  for (int i = threadIdx.x; i < E * (kTM / 32); i += blockDim.x) (&smask[0][0])[i] = 0u;
-  if (threadIdx.x == 0) rf.ticket[blockIdx.x] = 0u;   // ready for the next call
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < kMaxGroupCtas; i += blockDim.x) rf.look[i] = 0ull;
-  __syncthreads();
-  if (row < T) {
-    // the token's top k over the tiles' lists: tiles in ascending expert
-    // ranges, each list best first with equal values in ascending index, so
-    // equal values arrive in ascending index
-    cnt = 0;
-    thr = 0.f;
-    for (int t = 0; t < ntiles; ++t) {
-      const size_t base = ((size_t)row * ntiles + t) * rf.k;
-      for (int p = 0; p < rf.k; ++p) {
-        const int e = __ldcg(rf.cand_i + base + p);
-        if (e >= 0) topk_insert(bv, bi, cnt, thr, rf.k, __ldcg(rf.cand_v + base + p), e);
-      }
-    }
-    // p_j = exp(l_j - l_0) / sum, the sum in selection order (as route_token)
-    float z[kFuseK];
-    float sum = 0.f;
-#pragma unroll
-    for (int p = 0; p < kFuseK; ++p)
-      if (p < rf.k) { z[p] = expf(bv[p] - bv[0]); sum += z[p]; }
-    const float inv = 1.0f / sum;
-#pragma unroll
-    for (int p = 0; p < kFuseK; ++p)
-      if (p < rf.k) {
-        rf.idx[(size_t)row * rf.k + p] = bi[p];
-        rf.pw[(size_t)row * rf.k + p] = z[p] * inv;
-        atomicOr(&smask[bi[p]][(row - m0) >> 5], 1u << (row & 31));
-      }
-  }
-  __syncthreads();
-  // every bitmap word of this tile's tokens, zero or not (no zeroing pass)
-  const int w0 = m0 >> 5;
-  for (int i = threadIdx.x; i < E * (kTM / 32); i += blockDim.x) {
-    const int e = i / (kTM / 32), wq = i - e * (kTM / 32);
-    if (w0 + wq < rf.W) rf.bitmap[(size_t)e * rf.W + w0 + wq] = smask[e][wq];
   }
 }
 

@@ -148,20 +148,13 @@ int rl_moe_router_logits(const void* x, const void* w_router, int T, int H, int 
                          void* stream);
 
 /* Workspace bytes of rl_moe_prefill_router_ws (the layer's workspace plus
- * the router's scratch: the [T, E] fp32 logits, or the per-tile candidate
- * lists of the fused routing); 0 on a bad argument. */
+ * the [T, E] fp32 logits); 0 on a bad argument. */
 size_t rl_moe_router_workspace_bytes(int fmt, int T, int H, int I, int E, int k);
 
-/* The layer from x and the router weights (same arguments as
- * rl_moe_prefill_ws, with w_router in place of router_logits): the router
- * GEMM of rl_moe_router_logits, then the layer on its fp32 logits.  With
- * k <= 16 the exact top-k ("Red Lite dev72 - bounded verify, profiling",
- * section 1: per-row selection, same tie rule as rl_moe_route) runs in the
- * router launch's epilogue on the logits in registers, and the routing
- * launch is skipped; the selections and weights equal those of
- * rl_moe_route on the logits rl_moe_router_logits returns, bit for bit.
- * Device status as for rl_moe_prefill_ws (this call clears it at its
- * start). */
+/* The layer from x and the router weights: rl_moe_router_logits into the
+ * workspace, then rl_moe_prefill_ws on those logits (same arguments, with
+ * w_router in place of router_logits).  Device status as for
+ * rl_moe_prefill_ws (this call clears it at its start). */
 int rl_moe_prefill_router_ws(const void* x, const void* w_router, const void* const* expert_blobs,
                              int fmt, int T, int H, int I, int E, int k, float* y, void* workspace,
                              size_t ws_bytes, void* stream);

@@ -119,15 +119,15 @@ def _ws_routing(ws, T, E, k):
 @pytest.mark.parametrize("T,H,I,E,k,ties", [
     (2048, 2048, 512, 512, 10, False),     # the headline shapes
     (100, 160, 96, 40, 8, False),          # one partial expert tile
-    (5, 2048, 512, 1024, 16, False),       # eight expert tiles, the largest fused k
+    (5, 2048, 512, 1024, 16, False),       # eight expert tiles
     (300, 256, 256, 300, 6, True),         # equal logits across expert tiles (duplicated router rows)
-    (64, 256, 256, 64, 17, False),         # k above the fused limit: logits, then the routing launch
+    (64, 256, 256, 64, 17, False),         # k of 17
 ])
-def test_fused_routing_equals_routing_the_exported_logits(T, H, I, E, k, ties):
-    """The layer from x and W_r routes in the router launch's epilogue (k <=
-    16): its selections, weights, grouping and y equal, bit for bit, those of
-    rl_moe_route and rl_moe_prefill_ws on the logits rl_moe_router_logits
-    returns for the same x and W_r."""
+def test_layer_from_x_equals_routing_the_exported_logits(T, H, I, E, k, ties):
+    """The layer from x and W_r: its selections, weights, grouping and y
+    equal, bit for bit, those of rl_moe_route and rl_moe_prefill_ws on the
+    logits rl_moe_router_logits returns for the same x and W_r (ties across
+    expert tiles included: the lower expert index first)."""
     wl = synth.Workload("fused", T, H, I, E, k, synth.FMT_Q2)
     inp = synth.make_inputs(wl, seed=23)
     w = synth.router_weights(E, H, seed=24)
