@@ -234,13 +234,13 @@ int make_act_map(CUtensorMap* map, const void* base, int K, long long rows, int 
   return RL_OK;
 }
 
-// bf16 [rows][K] row-major, 128-byte swizzled boxes of 64 x 128 (router GEMM operands).
-int make_bf16_map(CUtensorMap* map, const void* base, int K, long long rows) {
+// bf16 [rows][K] row-major, 128-byte swizzled boxes of 64 x box_rows (router GEMM operands).
+int make_bf16_map(CUtensorMap* map, const void* base, int K, long long rows, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(RL_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {64u, 128u};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
   const cuuint32_t es[2] = {1u, 1u};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -262,9 +262,9 @@ int launch_router(const void* x, const void* wr, int T, int H, int E, float* log
     configured.fetch_or(bit, std::memory_order_release);
   }
   alignas(64) CUtensorMap xmap, wmap;
-  int rc = make_bf16_map(&xmap, x, H, T);
+  int rc = make_bf16_map(&xmap, x, H, T, rl::router::kTM);
   if (rc != RL_OK) return rc;
-  rc = make_bf16_map(&wmap, wr, H, E);
+  rc = make_bf16_map(&wmap, wr, H, E, rl::router::kTN);
   if (rc != RL_OK) return rc;
   const dim3 grid((T + rl::router::kTM - 1) / rl::router::kTM, (E + rl::router::kTN - 1) / rl::router::kTN);
   const cudaError_t e = rl::launch_k(rl::router::router_gemm_kernel, grid, dim3(rl::router::kThreads),

@@ -10,10 +10,10 @@
 // fp32 logits (4 MB at 2,048 tokens x 512 experts, kept in L2) feed the exact
 // top-k of step 1 in the same call.
 //
-// One CTA computes a 128-token x 128-expert tile: A = x rows (M = tokens),
+// One CTA computes a 128-token x 64-expert tile: A = x rows (M = tokens),
 // B = W_r rows (N = experts), both K-major and brought by TMA into the
 // 128-byte-swizzled layout, four 64-value K stages in flight; the fp32
-// accumulator lives in TMEM (128 columns).  Warp 0 lane 0 issues the loads,
+// accumulator lives in TMEM (64 columns).  Warp 0 lane 0 issues the loads,
 // warp 1 issues the MMAs (one elected lane), and all four warps read the
 // accumulator back (lane = token) and write the logits.  Every wait is
 // bounded; on timeout the CTA sets RL_DEV_WAIT_TIMEOUT, waits for its own
@@ -26,7 +26,7 @@ namespace rl {
 namespace router {
 
 constexpr int kTM = 128;                 // tokens per CTA (MMA M)
-constexpr int kTN = 128;                 // experts per CTA (MMA N)
+constexpr int kTN = 64;                  // experts per CTA (MMA N): 128 CTAs at 2,048 x 512
 constexpr int kTK = 64;                  // K values per stage: one 128-byte swizzled row of bf16
 constexpr int kStages = 4;
 constexpr int kABytes = kTM * 128;
