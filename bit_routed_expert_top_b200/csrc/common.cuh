@@ -35,6 +35,7 @@ template <> struct Fmt<RL_FMT_Q2> {
   static constexpr int kBits = 2;
   static constexpr int kPerByte = 4;
   static constexpr int kGroup = 16;        // values per code word = K-permutation group
+  static constexpr int kStripe = 2;        // values that share one bit position of the word's 16-bit halves
 };
 // Q1: 1-bit codes, 8 per byte, 32 per word; byte 5 holds the shift flags.
 template <> struct Fmt<RL_FMT_Q1> {
@@ -43,24 +44,29 @@ template <> struct Fmt<RL_FMT_Q1> {
   static constexpr int kBits = 1;
   static constexpr int kPerByte = 8;
   static constexpr int kGroup = 32;
+  static constexpr int kStripe = 4;        // values that share one bit position of the word's bytes
 };
 
 // K permutation shared by the decoded weights (A operand) and the staged
-// activations (B operand).  The decoder turns one 32-bit code word
-// (kGroup consecutive values) into kGroup/2 fp16x2 words; word c, half h
-// holds the value pi(2c+h) of the group, with
-//     pi(i) = (i >> 2) + kPerByte * (i & 3).
-// A dot product is unchanged by a K permutation applied to both operands, so
-// x (and h for the down projection) are stored with the same permutation:
-// position i of a group holds natural value pi(i).
+// activations (B operand).  The decoder turns one 32-bit code word (kGroup
+// consecutive values) into kGroup/2 fp16x2 words, taking together the kStripe
+// codes that sit at the same bit position of the word's 16-bit halves (Q2)
+// or bytes (Q1); position i of the group holds the value
+//     pi(i) = i / kStripe + 8 * (i % kStripe)
+// (8 = codes per 16-bit half for Q2, per byte for Q1).  A dot product is
+// unchanged by a K permutation applied to both operands, so x (and h for the
+// down projection) are stored with the same permutation: position i of a
+// group holds natural value pi(i).
 template <int FMT>
 __host__ __device__ __forceinline__ int perm_value(int i) {
-  return (i >> 2) + Fmt<FMT>::kPerByte * (i & 3);
+  constexpr int S = Fmt<FMT>::kStripe;
+  return i / S + 8 * (i % S);
 }
 // Inverse: natural value v of a group sits at position perm_pos(v).
 template <int FMT>
 __host__ __device__ __forceinline__ int perm_pos(int v) {
-  return 4 * (v % Fmt<FMT>::kPerByte) + v / Fmt<FMT>::kPerByte;
+  constexpr int S = Fmt<FMT>::kStripe;
+  return S * (v % 8) + v / 8;
 }
 template <int FMT>
 __host__ __device__ __forceinline__ int perm_pos_k(int k) {

@@ -1,7 +1,7 @@
 // gemm_simt.cuh - plain CUDA-core decode-GEMMs for steps 3 and 4.
 //
-// Same inputs, outputs and roundings as the tensor-core kernels (weights
-// rounded once to fp16, fp16 activations, fp32 sums, fp16 h and o), written
+// Same inputs, outputs and roundings as the tensor-core kernels (fp16
+// weights, fp16 activations, fp32 sums, fp16 h and o), written
 // as one thread per weight row with no tensor cores.  Used to cross-check the
 // tensor-core kernels stage by stage (rl_moe_debug_set_gemm) and nowhere on
 // the default path.
@@ -11,9 +11,10 @@
 
 namespace rl {
 
-// The 32 weights of sub-block sb (values 32*sb .. 32*sb+31 of the row), each
-// rounded once to fp16: d*(2s+1) and its product with the code are exact in
-// fp32, so the single rounding is the fp16 conversion.
+// The 32 weights of sub-block sb (values 32*sb .. 32*sb+31 of the row) as the
+// tensor-core decoders round them.  m = d*(2s+1) is exact in fp32.  Q2: the
+// scale is rounded to fp16 (M) and M(2u-3), exact in fp32, once more.  Q1:
+// m((2b-1)+delta), exact in fp32, is rounded once.
 template <int FMT>
 __device__ __forceinline__ void decode_sub_simt(const uint8_t* __restrict__ row, int sb,
                                                 float out[kSubVals]) {
@@ -24,11 +25,12 @@ __device__ __forceinline__ void decode_sub_simt(const uint8_t* __restrict__ row,
   const uint32_t S = (uint32_t)blk[2] | ((uint32_t)blk[3] << 8) | ((uint32_t)blk[4] << 16);
   const float m = dd * (float)(2 * ((S >> (3 * i)) & 7u) + 1);
   if constexpr (FMT == RL_FMT_Q2) {
+    const float M = __half2float(__float2half_rn(m));
 #pragma unroll
     for (int v = 0; v < kSubVals; ++v) {
       const int vv = i * kSubVals + v;
       const int u = (blk[5 + (vv >> 2)] >> (2 * (vv & 3))) & 3;
-      out[v] = __half2float(__float2half_rn(m * (float)(2 * u - 3)));
+      out[v] = __half2float(__float2half_rn(M * (float)(2 * u - 3)));
     }
   } else {
     const float delta = ((blk[5] >> i) & 1) ? 0.125f : -0.125f;

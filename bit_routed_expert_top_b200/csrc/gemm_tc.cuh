@@ -363,20 +363,30 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
 }
 
 // ------------------------------------------------------------ decoding ---
-// fp16 LUT of one sub-block.  Q2: bytes 2u, 2u+1 of (lo, hi) hold
-// fp16(d(2s+1)(2u-3)), u = 0..3; Q1: bytes 2b, 2b+1 of lo hold
-// fp16(d(2s+1)((2b-1)+delta)).  d(2s+1) and its product with the code are
-// exact in fp32, so each weight is rounded exactly once.
+// Sub-block scale m = d(2s+1), exact in fp32 (s as an exact float from the
+// 2^23 bit pattern).
+__device__ __forceinline__ float sub_scale(float dd, uint32_t S, int i) {
+  const float sf = __uint_as_float(0x4B000000u | ((S >> (3 * i)) & 7u)) - 8388608.0f;
+  return fmaf(sf, 2.0f * dd, dd);
+}
+
+// fp16 LUT of one sub-block.
+// Q2: bytes 2u, 2u+1 of (lo, hi) hold the weight of code u = 0..3,
+//     fp16(M(2u-3)) with M = fp16(m): the scale is rounded to fp16 once and
+//     its product with the odd code value once more (exactly what the
+//     fused multiply-add decode below computes, so both decoders give every
+//     code the same weight).
+// Q1: bytes 2b, 2b+1 of lo hold fp16(m((2b-1)+delta)), rounded once (the
+//     product is exact in fp32).
 template <int FMT>
 __device__ __forceinline__ void make_lut(float dd, uint32_t S, uint32_t flags, int i, uint32_t& lo,
                                          uint32_t& hi) {
-  // s as an exact float from the 2^23 bit pattern, then m = d(2s+1) (exact)
-  const float sf = __uint_as_float(0x4B000000u | ((S >> (3 * i)) & 7u)) - 8388608.0f;
-  const float m = fmaf(sf, 2.0f * dd, dd);
+  const float m = sub_scale(dd, S, i);
   if constexpr (FMT == RL_FMT_Q2) {
-    const __half2 p = __floats2half2_rn(m, 3.0f * m);          // u=2 (low), u=3 (high)
-    hi = *reinterpret_cast<const uint32_t*>(&p);
-    lo = __byte_perm(hi, 0u, 0x1032) ^ 0x80008000u;            // u=0: -3m, u=1: -m
+    const __half2 p = __float2half2_rn(m);                     // (M, M)
+    const uint32_t pb = *reinterpret_cast<const uint32_t*>(&p);
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(pb), "r"(0x42003C00u));   // u=2: M*1, u=3: M*3
+    lo = __byte_perm(hi, 0u, 0x1032) ^ 0x80008000u;            // u=0: -3M, u=1: -M
   } else {
     const float delta = ((flags >> i) & 1u) ? 0.125f : -0.125f;
     const __half2 p = __floats2half2_rn(m * (delta - 1.0f), m * (delta + 1.0f));
@@ -385,16 +395,15 @@ __device__ __forceinline__ void make_lut(float dd, uint32_t S, uint32_t flags, i
   }
 }
 
-// One 32-bit code word -> fp16x2 words out[0 .. G/2).  Word 2k+h holds the
-// values (k + 2h*P, k + (2h+1)*P) of the group, P = codes per byte, i.e.
-// position i holds value (i >> 2) + P*(i & 3).
-//
-// Per four codes: the selectors of bytes 0-1 as one multiply-add on the FMA
-// pipe; the shift, the mask, the selectors of bytes 2-3 (a byte permute of
-// the first selector word) and the two table permutes on the integer ALU
-// pipe.  Measured against a mad.hi for the second selector, which compiles
-// to two instructions, this takes ~11% fewer instructions per code word; a
-// high multiply in place of the shift measured slower.
+// Q2 scale pair of one sub-block for decode_word_fma: M1 = (M, M), M2 = 2*M1
+// (exact), M = fp16(m).
+__device__ __forceinline__ void make_scale_pair(float dd, uint32_t S, int i, uint32_t& m1, uint32_t& m2) {
+  const __half2 p = __float2half2_rn(sub_scale(dd, S, i));
+  const __half2 q = __hadd2(p, p);
+  m1 = *reinterpret_cast<const uint32_t*>(&p);
+  m2 = *reinterpret_cast<const uint32_t*>(&q);
+}
+
 // Byte permute with the hardware's selector semantics.  __byte_perm keeps
 // only 3 bits of each selector nibble, so with a selector that is not a
 // compile-time constant it costs a masking instruction before the permute;
@@ -404,20 +413,93 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
   return r;
 }
+
+// One 32-bit code word -> fp16x2 words out[0 .. G/2) through the LUT, in the
+// K order of perm_value: output word w holds the kStripe codes at one bit
+// position of the 16-bit halves (Q2: codes w, w+8) or of the bytes (Q1:
+// word 2k+h holds codes k + 16h, k + 16h + 8).
+//
+// Per four codes: the selectors of bytes 0-1 as one multiply-add on the FMA
+// pipe; the shift, the mask, the selectors of bytes 2-3 (a byte permute of
+// the first selector word) and the two table permutes on the integer ALU
+// pipe.  Q2 first swaps bytes 1 and 2 of the word, so that each selector
+// word pairs a code of the low half with the code at the same position of
+// the high half.
 template <int FMT>
 __device__ __forceinline__ void decode_word(uint32_t c, uint32_t lo, uint32_t hi, uint32_t* out) {
   constexpr int P = Fmt<FMT>::kPerByte;
   constexpr int B = Fmt<FMT>::kBits;
   constexpr uint32_t mask = FMT == RL_FMT_Q2 ? 0x03030303u : 0x01010101u;
+  if constexpr (FMT == RL_FMT_Q2) c = __byte_perm(c, 0u, 0x3120u);
 #pragma unroll
   for (int k = 0; k < P; ++k) {
     const uint32_t shifted = c >> (B * k);
     const uint32_t v = shifted & mask;
     const uint32_t sel_lo = v * 0x22u + 0x10101010u;          // selectors of bytes 0-1
     const uint32_t sel_hi = __byte_perm(sel_lo, 0u, 0x3232u);     // selectors of bytes 2-3
-    out[2 * k] = prmt(lo, hi, sel_lo);
-    out[2 * k + 1] = prmt(lo, hi, sel_hi);
+    if constexpr (FMT == RL_FMT_Q2) {
+      out[k] = prmt(lo, hi, sel_lo);                             // codes k, k+8
+      out[k + 4] = prmt(lo, hi, sel_hi);                         // codes k+4, k+12
+    } else {
+      out[2 * k] = prmt(lo, hi, sel_lo);
+      out[2 * k + 1] = prmt(lo, hi, sel_hi);
+    }
   }
+}
+
+// Q2 code word -> the same eight fp16x2 words as decode_word, by fp16
+// arithmetic instead of table permutes.  For the code pair at bit 2j of both
+// 16-bit halves, OR-ing the masked bits into the fp16 pattern of 1024 gives
+// 1024 + 4^j c exactly (the bits land in the mantissa, whose unit is 1 in
+// [1024, 2048)); one fused multiply-add by 4^-j, minus 1024 * 4^-j + 2,
+// gives c - 2 exactly, and a second, (c - 2) * 2M + M, the weight M(2c - 3)
+// rounded once.  Codes at bits 10-15 of each half come from the word
+// shifted right by 10.  One integer instruction and two fp16x2 multiply-adds
+// per two codes: the decoders mix this form with the table form to balance
+// the ALU and FMA pipes.
+struct Fp16Consts {
+  uint32_t magic, scale[5], offset[5];
+};
+__device__ __forceinline__ Fp16Consts fp16_consts() {
+  // 4^-j and -(1024 * 4^-j + 2) as fp16 pairs, j = 0..4, and 1024; moved
+  // through an opaque register so they stay in registers for the whole loop
+  const uint32_t sc[5] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u, 0x1C001C00u};
+  const uint32_t of[5] = {0xE402E402u, 0xDC08DC08u, 0xD420D420u, 0xCC80CC80u, 0xC600C600u};
+  Fp16Consts k;
+#pragma unroll
+  for (int j = 0; j < 5; ++j) {
+    asm volatile("mov.b32 %0, %1;" : "=r"(k.scale[j]) : "r"(sc[j]));
+    asm volatile("mov.b32 %0, %1;" : "=r"(k.offset[j]) : "r"(of[j]));
+  }
+  asm volatile("mov.b32 %0, %1;" : "=r"(k.magic) : "r"(0x64006400u));
+  return k;
+}
+template <int J>
+__device__ __forceinline__ uint32_t code_pair_bits(uint32_t src, uint32_t magic) {
+  uint32_t r;   // (src & pair mask) | magic
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(src), "n"(0x00030003u << (2 * J)), "r"(magic));
+  return r;
+}
+__device__ __forceinline__ uint32_t hfma2_bits(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+template <int J>
+__device__ __forceinline__ uint32_t decode_pair_fma(uint32_t src, uint32_t m2, uint32_t m1, const Fp16Consts& k) {
+  return hfma2_bits(hfma2_bits(code_pair_bits<J>(src, k.magic), k.scale[J], k.offset[J]), m2, m1);
+}
+__device__ __forceinline__ void decode_word_fma(uint32_t c, uint32_t m1, uint32_t m2, const Fp16Consts& k,
+                                                uint32_t* out) {
+  const uint32_t c10 = c >> 10;
+  out[0] = decode_pair_fma<0>(c, m2, m1, k);
+  out[1] = decode_pair_fma<1>(c, m2, m1, k);
+  out[2] = decode_pair_fma<2>(c, m2, m1, k);
+  out[3] = decode_pair_fma<3>(c, m2, m1, k);
+  out[4] = decode_pair_fma<4>(c, m2, m1, k);
+  out[5] = decode_pair_fma<0>(c10, m2, m1, k);
+  out[6] = decode_pair_fma<1>(c10, m2, m1, k);
+  out[7] = decode_pair_fma<2>(c10, m2, m1, k);
 }
 
 // 8 bytes starting at byte offset o of a shared-memory row region (o may be
@@ -759,6 +841,7 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
     // the global step index ring_it of the current unit's step 0.
     int rs = 0;
     uint32_t rpar = 0, ring_it = 0;
+    const Fp16Consts fk = fp16_consts();
     for (int ui = 0; ui < my_units && ok; ++ui) {
       // this thread's row (block 0) of the unit: the offset of a block inside
       // its 16-byte aligned copy follows from it, block by block
@@ -807,15 +890,22 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               const int i = i0 + 2 * hh;        // first sub-block of this half
-              uint32_t lo0, hi0, lo1, hi1;
-              make_lut<FMT>(dd, S, flags, i, lo0, hi0);
-              make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
               if constexpr (FMT == RL_FMT_Q2) {
+                // one code word in four through the table (ALU pipe), three
+                // by fp16 multiply-adds (FMA pipe): the two pipes about
+                // equally loaded
+                uint32_t lo0, hi0, m1a, m2a, m1b, m2b;
+                make_lut<FMT>(dd, S, flags, i, lo0, hi0);
+                make_scale_pair(dd, S, i, m1a, m2a);
+                make_scale_pair(dd, S, i + 1, m1b, m2b);
                 decode_word<FMT>(cw[hh][0], lo0, hi0, words);
-                decode_word<FMT>(cw[hh][1], lo0, hi0, words + 8);
-                decode_word<FMT>(cw[hh][2], lo1, hi1, words + 16);
-                decode_word<FMT>(cw[hh][3], lo1, hi1, words + 24);
+                decode_word_fma(cw[hh][1], m1a, m2a, fk, words + 8);
+                decode_word_fma(cw[hh][2], m1b, m2b, fk, words + 16);
+                decode_word_fma(cw[hh][3], m1b, m2b, fk, words + 24);
               } else {
+                uint32_t lo0, hi0, lo1, hi1;
+                make_lut<FMT>(dd, S, flags, i, lo0, hi0);
+                make_lut<FMT>(dd, S, flags, i + 1, lo1, hi1);
                 decode_word<FMT>(cw[hh][0], lo0, hi0, words);
                 decode_word<FMT>(cw[hh][1], lo1, hi1, words + 16);
               }

@@ -59,7 +59,7 @@ __device__ __forceinline__ uint32_t ldg_u32_at(const uint8_t* p) {
 // Dot product of one block (256 values of a row, at byte address blk) with
 // 256 activations xs2 held as fp16x2 words in the decoder's K order (word w
 // = the two values decode_word puts in its output word w).  Every weight is
-// rounded once to fp16 exactly as the tensor-core decoders round it; the 16
+// rounded to fp16 exactly as the tensor-core decoders round it; the 16
 // products of a code word are summed in fp16x2 (8 fused multiply-adds per
 // half), each code word's partial then in fp32.
 template <int FMT>

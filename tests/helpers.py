@@ -44,15 +44,15 @@ def to_device(inp, device="cuda"):
 
 def unpermute_k(a, fmt):
     """Undo the per-group K permutation of the library's fp16 staging buffers
-    (position i of a group of G holds natural value (i>>2) + (G/4)*(i&3)), so
-    the library's h can be compared with the oracle's.  Test-side restatement
-    of the documented buffer layout."""
-    G = 16 if fmt == synth.FMT_Q2 else 32
-    per_byte = G // 4
+    (groups of G = 16 values for Q2, 32 for Q1; position i of a group holds
+    natural value i // S + 8 * (i % S), S = 2 for Q2 and 4 for Q1), so the
+    library's h can be compared with the oracle's.  Test-side restatement of
+    the documented buffer layout."""
+    G, S = (16, 2) if fmt == synth.FMT_Q2 else (32, 4)
     a = np.asarray(a)
     K = a.shape[-1]
     out = np.empty_like(a)
     for g0 in range(0, K, G):
         for i in range(G):
-            out[..., g0 + (i >> 2) + per_byte * (i & 3)] = a[..., g0 + i]
+            out[..., g0 + i // S + 8 * (i % S)] = a[..., g0 + i]
     return out
