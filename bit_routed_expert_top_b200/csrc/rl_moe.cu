@@ -341,22 +341,22 @@ int launch_small(const void* x, const float* logits, const rl::ExpertTable& tab,
   const bool prof = g_prof.load(std::memory_order_relaxed);
   const bool pdl = !prof;
   mark(0, s);
-  const int per = (d.E + 31) / 32;
-  const dim3 rg((d.T + 7) / 8), rb(rl::small::kThreads);
-  if (per <= 1) rl::small::route_small_kernel<1><<<rg, rb, 0, s>>>(logits, d, w);
-  else if (per <= 2) rl::small::route_small_kernel<2><<<rg, rb, 0, s>>>(logits, d, w);
-  else if (per <= 4) rl::small::route_small_kernel<4><<<rg, rb, 0, s>>>(logits, d, w);
-  else if (per <= 8) rl::small::route_small_kernel<8><<<rg, rb, 0, s>>>(logits, d, w);
-  else if (per <= 16) rl::small::route_small_kernel<16><<<rg, rb, 0, s>>>(logits, d, w);
-  else rl::small::route_small_kernel<32><<<rg, rb, 0, s>>>(logits, d, w);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "route_small_kernel launch");
   mark(1, s);
   mark(2, s);
+  // launch 1 (routing + gate/up) is a plain launch: it starts once the
+  // previous call's kernels have finished with h and the routing buffers
+  const int per = (d.E + 31) / 32;
   const int rows_c = 4 * (32 / d.nbH);
   const size_t smem = (size_t)d.nbH * rl::small::kSliceW * sizeof(__half2);
-  e = rl::launch_k(rl::small::gateup_small_kernel<FMT>, dim3(d.P, (d.I + rows_c - 1) / rows_c),
-                   dim3(rl::small::kThreads), smem, s, pdl, static_cast<const uint16_t*>(x), d, w, tab, h32);
+  const dim3 g1(d.P, (d.I + rows_c - 1) / rows_c), b1(rl::small::kThreads);
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  if (per <= 1) rl::small::gateup_small_kernel<FMT, 1><<<g1, b1, smem, s>>>(xb, logits, d, w, tab, h32);
+  else if (per <= 2) rl::small::gateup_small_kernel<FMT, 2><<<g1, b1, smem, s>>>(xb, logits, d, w, tab, h32);
+  else if (per <= 4) rl::small::gateup_small_kernel<FMT, 4><<<g1, b1, smem, s>>>(xb, logits, d, w, tab, h32);
+  else if (per <= 8) rl::small::gateup_small_kernel<FMT, 8><<<g1, b1, smem, s>>>(xb, logits, d, w, tab, h32);
+  else if (per <= 16) rl::small::gateup_small_kernel<FMT, 16><<<g1, b1, smem, s>>>(xb, logits, d, w, tab, h32);
+  else rl::small::gateup_small_kernel<FMT, 32><<<g1, b1, smem, s>>>(xb, logits, d, w, tab, h32);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gateup_small_kernel launch");
   mark(3, s);
   const size_t smem2 = (size_t)d.k * d.nbI * rl::small::kSliceW * sizeof(__half2);

@@ -154,7 +154,7 @@ DECODE_REGIME = [
 
 @pytest.mark.parametrize("wl", DECODE_REGIME, ids=lambda w: w.name)
 def test_decode_regime_every_output_and_against_the_prefill_path(wl):
-    """Chunks of at most 64 pairs whose shapes fit it take the three-launch
+    """Chunks of at most 64 pairs whose shapes fit it take the two-launch
     decode-regime path: every output against the oracle, the routing it
     publishes bit for bit, and the same inputs forced through the six-launch
     prefill path (both within the layer's tolerance of the oracle)."""
