@@ -60,7 +60,7 @@ namespace tc {
 #define RL_TC_RAW_STAGES 4
 #endif
 #ifndef RL_TC_B_STAGES
-#define RL_TC_B_STAGES 4
+#define RL_TC_B_STAGES 6
 #endif
 #ifndef RL_TC_DEC_PHASES
 #define RL_TC_DEC_PHASES 2
@@ -455,8 +455,11 @@ __device__ __forceinline__ void decode_word(uint32_t c, uint32_t lo, uint32_t hi
 // gives c - 2 exactly, and a second, (c - 2) * 2M + M, the weight M(2c - 3)
 // rounded once.  Codes at bits 10-15 of each half come from the word
 // shifted right by 10.  One integer instruction and two fp16x2 multiply-adds
-// per two codes: the decoders mix this form with the table form to balance
-// the ALU and FMA pipes.
+// per two codes, against about three integer instructions for the table
+// form: the tensor-core decoders use this form for every Q2 word (their
+// integer pipe also carries the step's index and load arithmetic), the
+// decode-regime dot products one word in two (their fp16 multiply-adds
+// already load the FMA pipe).
 struct Fp16Consts {
   uint32_t magic, scale[5], offset[5];
 };
@@ -891,14 +894,14 @@ decode_gemm_kernel(Dims d, Work w, ExpertTable tab, const __grid_constant__ CUte
             for (int hh = 0; hh < 2; ++hh) {
               const int i = i0 + 2 * hh;        // first sub-block of this half
               if constexpr (FMT == RL_FMT_Q2) {
-                // one code word in four through the table (ALU pipe), three
-                // by fp16 multiply-adds (FMA pipe): the two pipes about
-                // equally loaded
-                uint32_t lo0, hi0, m1a, m2a, m1b, m2b;
-                make_lut<FMT>(dd, S, flags, i, lo0, hi0);
+                // every code word by fp16 multiply-adds (measured against
+                // one word in four through the table: the same gate/up time,
+                // down 113.7 -> 110.6 us; the integer pipe also carries the
+                // step's index and load arithmetic)
+                uint32_t m1a, m2a, m1b, m2b;
                 make_scale_pair(dd, S, i, m1a, m2a);
                 make_scale_pair(dd, S, i + 1, m1b, m2b);
-                decode_word<FMT>(cw[hh][0], lo0, hi0, words);
+                decode_word_fma(cw[hh][0], m1a, m2a, fk, words);
                 decode_word_fma(cw[hh][1], m1a, m2a, fk, words + 8);
                 decode_word_fma(cw[hh][2], m1b, m2b, fk, words + 16);
                 decode_word_fma(cw[hh][3], m1b, m2b, fk, words + 24);
