@@ -33,9 +33,11 @@
  * matrix with K columns is ceil(K/256) consecutive blocks (values past K are
  * ignored).  Bytes per expert: rl_moe_expert_bytes().
  *
- * Arithmetic: decoded weights are rounded once to fp16, x (bf16) is converted
- * to fp16, products accumulate in fp32 on the tensor cores, h is stored as
- * fp16, o as fp16, the combine runs in fp32.  y is fp32.
+ * Arithmetic: decoded weights are fp16 (Q1: d(2s+1)((2b-1)+delta) rounded
+ * once; Q2: the sub-block scale d(2s+1) rounded to fp16, M, then M(2u-3)
+ * rounded, so +-M exactly), x (bf16) is converted to fp16, products
+ * accumulate in fp32 on the tensor cores, h is stored as fp16, o as fp16,
+ * the combine runs in fp32.  y is fp32.
  *
  * Conventions for every entry point:
  *   - Device pointers are CUDA global memory on the current device; host
