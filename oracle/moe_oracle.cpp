@@ -355,6 +355,25 @@ int orc_moe_prefill_tokens(int fmt, const uint16_t* x_rows, const float* logit_r
   return 0;
 }
 
+// Shared expert: y[t] += o_s[t] for every token t, o_s[t] the FFN (ffn_row)
+// of one more expert blob of the same format and shape applied to x_t with
+// weight 1, added after the routed sum.  "Red Lite dev75 - --kv f16, faster
+// prompt ingestion", section 2, lists a shared expert beside the routed
+// experts in the prefill (dense: every token, no routing); the pages give no
+// gate for it, so none is applied.  x_bits bf16 [T,H]; y [T,H] in and out.
+int orc_shared_expert_add(int fmt, const uint16_t* x_bits, const uint8_t* blob, int T, int H, int I, double* y) {
+  if (!dims_ok(fmt, H, I) || T < 0 || (T && (!x_bits || !blob || !y))) return -1;
+  Expert ex;
+  if (T) decode_expert(fmt, blob, H, I, &ex);
+  std::vector<double> x((size_t)H), hrow((size_t)I), orow((size_t)H);
+  for (int t = 0; t < T; ++t) {
+    for (int c = 0; c < H; ++c) x[c] = bf16_to_double(x_bits[(size_t)t * H + c]);
+    ffn_row(ex.wg.data(), ex.wu.data(), ex.wd.data(), H, I, x.data(), hrow.data(), orow.data());
+    for (int c = 0; c < H; ++c) y[(size_t)t * H + c] += orow[c];
+  }
+  return 0;
+}
+
 unsigned orc_hardware_concurrency() { return std::thread::hardware_concurrency(); }
 
 }  // extern "C"

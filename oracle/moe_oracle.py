@@ -64,6 +64,7 @@ _SIGNATURES = {
     "orc_moe_prefill_tokens": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
     "orc_expert_outputs": (_i, [_i, _p, _p, _i, _i, _i, _i, _i, _p, _p, _i, _i, _p]),
     "orc_router_logits": (_i, [_p, _p, _i, _i, _i, _p]),
+    "orc_shared_expert_add": (_i, [_i, _p, _p, _i, _i, _i, _p]),
     "orc_hardware_concurrency": (ctypes.c_uint, []),
 }
 
@@ -260,6 +261,22 @@ def moe_prefill(x_bits, logits, blobs, fmt: int, H: int, I: int, k: int,
     if keep_intermediates:
         out["h"] = h
         out["o"] = o
+    return out
+
+
+def shared_expert_add(x_bits, blob, fmt: int, H: int, I: int, y):
+    """y [T, H] float64 plus, per token, the FFN of the shared expert's blob
+    applied to its x row with weight 1 (added after the routed sum).
+    Returns a new array; y is not modified."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    T = x_bits.shape[0]
+    out = np.array(y, dtype=np.float64, copy=True, order="C")
+    if x_bits.shape != (T, H) or out.shape != (T, H):
+        raise ValueError("inconsistent shapes")
+    b = np.ascontiguousarray(blob, dtype=np.uint8)
+    if b.size < expert_bytes(fmt, H, I):
+        raise ValueError("shared expert blob too short")
+    _check(load().orc_shared_expert_add(fmt, _ptr(x_bits), _ptr(b), T, H, I, _ptr(out)), "shared_expert_add")
     return out
 
 

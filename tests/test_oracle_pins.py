@@ -393,3 +393,59 @@ def test_pages_figures_headline_chunk():
     assert offsets[-1] / wl.E == pytest.approx(fig["pairs_per_expert"]["value"], rel=0.05)
     dense_f32 = wl.E * 3 * wl.H * wl.I * 4
     assert dense_f32 == pytest.approx(fig["whole_expert_dequant_bytes"]["value"], rel=0.1)
+
+
+# ------------------------------------------------------------ shared expert ---
+
+def test_shared_expert_closed_form_constant_blob():
+    """Constant shared expert (gate a, up b, down c), x = 1: every token's
+    y row gains c*I*silu(a*H)*(b*H) in every column, on top of what it held."""
+    H, I, T = 256, 64, 3
+    a, b, c = 2.0 ** -10 * 3, 2.0 ** -9, 2.0 ** -6 * 3
+    blob = _blob(O.FMT_Q2, H, I, [_const_q2_block(2.0 ** -10, 3)] * I, [_const_q2_block(2.0 ** -9, 2)] * I,
+                 [_const_q2_block(2.0 ** -6, 3)] * H)
+    x = np.full((T, H), 0x3F80, np.uint16)
+    y0 = np.arange(T * H, dtype=np.float64).reshape(T, H) * 0.5      # exact in float64
+    y = O.shared_expert_add(x, blob, O.FMT_Q2, H, I, y0)
+    g = a * H
+    want = c * I * (g / (1 + math.exp(-g))) * (b * H)
+    np.testing.assert_allclose(y - y0, want, rtol=1e-13)
+    assert np.array_equal(y0, np.arange(T * H, dtype=np.float64).reshape(T, H) * 0.5)   # input untouched
+
+
+@pytest.mark.parametrize("fmt", [1, 2])
+def test_shared_expert_is_a_one_expert_layer_on_every_token(fmt):
+    """The shared expert added to zeros equals the routed layer with one
+    expert (that blob) and k = 1, where every token's single pick has
+    p = 1: the same FFN of every token, bit for bit."""
+    from bit_routed_expert_top_b200 import synth
+    wl = synth.Workload("t", 9, 96, 64, 1, 1, fmt)
+    inp = synth.make_inputs(wl, seed=31 + fmt)
+    nb = O.expert_bytes(fmt, wl.H, wl.I)
+    blob = inp.blobs[0, :nb]
+    routed = O.moe_prefill(inp.x_bits, inp.logits, [blob], fmt, wl.H, wl.I, 1)
+    assert np.all(routed["p"] == 1.0)
+    y = O.shared_expert_add(inp.x_bits, blob, fmt, wl.H, wl.I, np.zeros((wl.T, wl.H)))
+    assert np.array_equal(y, routed["y"])
+
+
+def test_shared_expert_dense_brute_force():
+    """Every token's shared-expert row from the decoded matrices by plain
+    loops (no library matrix product), added to a nonzero y."""
+    from bit_routed_expert_top_b200 import synth
+    wl = synth.Workload("t", 4, 96, 32, 1, 1, synth.FMT_Q2)
+    inp = synth.make_inputs(wl, seed=17)
+    nb = O.expert_bytes(wl.fmt, wl.H, wl.I)
+    blob = inp.blobs[0, :nb]
+    wg, wu, wd = O.expert_weights(blob, wl.fmt, wl.H, wl.I)
+    x = O.bf16_bits_to_f64(inp.x_bits)
+    y0 = np.random.default_rng(3).standard_normal((wl.T, wl.H))
+    want = y0.copy()
+    for t in range(wl.T):
+        g = [sum(wg[r, h] * x[t, h] for h in range(wl.H)) for r in range(wl.I)]
+        u = [sum(wu[r, h] * x[t, h] for h in range(wl.H)) for r in range(wl.I)]
+        hh = [g[r] / (1 + math.exp(-g[r])) * u[r] for r in range(wl.I)]
+        for c in range(wl.H):
+            want[t, c] += sum(wd[c, r] * hh[r] for r in range(wl.I))
+    y = O.shared_expert_add(inp.x_bits, blob, wl.fmt, wl.H, wl.I, y0)
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
