@@ -27,6 +27,8 @@ SIGNATURES = {
     "rl_moe_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "rl_moe_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp]),
     "rl_moe_prefill_ws": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "rl_moe_shared_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "rl_moe_prefill_shared_ws": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
     "rl_moe_prefill_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp]),
     "rl_moe_route": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "rl_moe_check_status": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_uint)]),
@@ -188,6 +190,33 @@ def rl_moe_prefill_ws(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, wor
     _check(load().rl_moe_prefill_ws(_ptr(x), _ptr(router_logits), ctypes.cast(table, ctypes.c_void_p),
                                     fmt, T, H, I, E, k, _ptr(y), _ptr(workspace), nbytes,
                                     _stream(stream)))
+
+
+def rl_moe_shared_workspace_bytes(fmt: int, T: int, H: int, I: int, E: int, k: int) -> int:
+    n = load().rl_moe_shared_workspace_bytes(fmt, T, H, I, E, k)
+    if n == 0:
+        raise RlMoeError(-1, load().rl_last_error().decode(errors="replace"))
+    return n
+
+
+def alloc_shared_workspace(fmt, T, H, I, E, k, device=None) -> torch.Tensor:
+    n = rl_moe_shared_workspace_bytes(fmt, T, H, I, E, k)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def rl_moe_prefill_shared_ws(x, router_logits, expert_blobs, shared_blob, fmt, T, H, I, E, k, y, workspace,
+                             stream=None):
+    """The layer plus a shared expert (one more blob, every token, weight 1,
+    added after the routed sum); see include/rl_moe.h."""
+    _check_layer_bufs(x, router_logits, y, T, H, E)
+    _check_buf(shared_blob, "shared_blob", (torch.uint8,), rl_moe_expert_bytes(fmt, H, I))
+    _check_buf(workspace, "workspace", (), 0)
+    _need_cuda(x, router_logits, y, workspace, shared_blob)
+    table = expert_blobs if isinstance(expert_blobs, ctypes.Array) else expert_table(expert_blobs, E)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().rl_moe_prefill_shared_ws(_ptr(x), _ptr(router_logits), ctypes.cast(table, ctypes.c_void_p),
+                                           _ptr(shared_blob), fmt, T, H, I, E, k, _ptr(y), _ptr(workspace),
+                                           nbytes, _stream(stream)))
 
 
 def rl_moe_prefill_noalloc(x, router_logits, expert_blobs, fmt, T, H, I, E, k, y, stream=None):

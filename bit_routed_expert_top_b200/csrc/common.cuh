@@ -84,6 +84,11 @@ struct ExpertTable {
 
 struct Dims {
   int T, H, I, E, k, fmt;
+  // E_route routed experts (logits per token), k_route picks among them; with
+  // a shared expert E = E_route + 1 (the shared one is expert E_route) and
+  // k = k_route + 1 (every token's last pick, weight 1), else E = E_route and
+  // k = k_route.
+  int E_route, k_route;
   int P;          // T * k pairs
   int W;          // ceil(T / 32) bitmap words per expert
   int nbH, nbI;   // blocks per row of gate/up (K=H) and down (K=I)

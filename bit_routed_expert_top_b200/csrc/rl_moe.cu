@@ -120,9 +120,15 @@ int check_dims(int fmt, int T, int H, int I, int E, int k) {
   return RL_OK;
 }
 
-int plan(int fmt, int T, int H, int I, int E, int k, rl::Dims* d, Layout* L) {
-  const int rc = check_dims(fmt, T, H, I, E, k);
+// shared = 1: one more expert (index E) that every token picks last with
+// weight 1; the pipeline then runs over E + 1 experts and k + 1 picks.
+int plan(int fmt, int T, int H, int I, int E, int k, rl::Dims* d, Layout* L, int shared = 0) {
+  const int rc = check_dims(fmt, T, H, I, E + shared, k + shared);
   if (rc != RL_OK) return rc;
+  d->E_route = E;
+  d->k_route = k;
+  E += shared;
+  k += shared;
   d->T = T; d->H = H; d->I = I; d->E = E; d->k = k; d->fmt = fmt;
   d->P = T * k;
   d->W = (T + 31) / 32;
@@ -311,7 +317,7 @@ long long uniform_expert_stride(const rl::ExpertTable& tab, const rl::Dims& d) {
 // values per lane = smallest power of two >= E/32.
 void launch_route(const float* logits, const rl::Dims& d, const rl::Work& w, cudaStream_t s) {
   const int grid = d.W * 4;
-  const int per = (d.E + 31) / 32;
+  const int per = (d.E_route + 31) / 32;
   if (per <= 1) rl::route_kernel<1><<<grid, 256, 0, s>>>(logits, d, w);
   else if (per <= 2) rl::route_kernel<2><<<grid, 256, 0, s>>>(logits, d, w);
   else if (per <= 4) rl::route_kernel<4><<<grid, 256, 0, s>>>(logits, d, w);
@@ -345,7 +351,7 @@ int launch_small(const void* x, const float* logits, const rl::ExpertTable& tab,
   mark(2, s);
   // launch 1 (routing + gate/up) is a plain launch: it starts once the
   // previous call's kernels have finished with h and the routing buffers
-  const int per = (d.E + 31) / 32;
+  const int per = (d.E_route + 31) / 32;
   const int rows_c = 4 * (32 / d.nbH);
   const size_t smem = (size_t)d.nbH * rl::small::kSliceW * sizeof(__half2);
   const dim3 g1(d.P, (d.I + rows_c - 1) / rows_c), b1(rl::small::kThreads);
@@ -489,6 +495,43 @@ int rl_moe_prefill_ws(const void* x, const float* router_logits, const void* con
   static thread_local rl::ExpertTable tab;
   rc = fill_table(expert_blobs, E, &tab);
   if (rc != RL_OK) return rc;
+  const rl::Work w = carve(workspace, L);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (small_path_fits(d, L)) {
+    float* h32 = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.h16);
+    return fmt == RL_FMT_Q2 ? launch_small<RL_FMT_Q2>(x, router_logits, tab, d, w, h32, y, s)
+                            : launch_small<RL_FMT_Q1>(x, router_logits, tab, d, w, h32, y, s);
+  }
+  return fmt == RL_FMT_Q2 ? launch_all<RL_FMT_Q2>(x, router_logits, tab, d, w, y, s)
+                          : launch_all<RL_FMT_Q1>(x, router_logits, tab, d, w, y, s);
+}
+
+size_t rl_moe_shared_workspace_bytes(int fmt, int T, int H, int I, int E, int k) {
+  rl::Dims d;
+  Layout L;
+  if (plan(fmt, T, H, I, E, k, &d, &L, 1) != RL_OK) return 0;
+  return L.total;
+}
+
+int rl_moe_prefill_shared_ws(const void* x, const float* router_logits, const void* const* expert_blobs,
+                             const void* shared_blob, int fmt, int T, int H, int I, int E, int k, float* y,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  rl::Dims d;
+  Layout L;
+  int rc = plan(fmt, T, H, I, E, k, &d, &L, 1);
+  if (rc != RL_OK) return rc;
+  if (T == 0) return RL_OK;
+  if (!x || !router_logits || !y || !workspace || !shared_blob)
+    return fail(RL_ERR_INVALID_ARG, "NULL x, router_logits, shared_blob, y or workspace");
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(y) % 16 ||
+      reinterpret_cast<uintptr_t>(workspace) % 256 || reinterpret_cast<uintptr_t>(shared_blob) % 16)
+    return fail(RL_ERR_INVALID_ARG, "x, y and shared_blob must be 16-byte aligned, workspace 256-byte aligned");
+  if (ws_bytes < L.total)
+    return fail(RL_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, L.total);
+  static thread_local rl::ExpertTable tab;
+  rc = fill_table(expert_blobs, E, &tab);
+  if (rc != RL_OK) return rc;
+  tab.p[E] = static_cast<const uint8_t*>(shared_blob);
   const rl::Work w = carve(workspace, L);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (small_path_fits(d, L)) {

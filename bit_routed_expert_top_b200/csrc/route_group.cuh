@@ -104,6 +104,16 @@ __device__ __forceinline__ void route_token(const float* __restrict__ row, int E
   for (int j = 32 + lane; j < k; j += 32) pw[j] *= inv;
 }
 
+// The shared expert as every token's last pick: expert E_route with weight
+// 1, after the k_route routed picks (so the combine adds it last).  "Red Lite
+// dev75 - --kv f16, faster prompt ingestion", section 2, lists a shared
+// expert beside the routed ones in the prefill; the pages give it no gate.
+__device__ __forceinline__ void append_shared(const Dims& d, int* idx, float* pw, unsigned* smask, int warp) {
+  idx[d.k_route] = d.E_route;
+  pw[d.k_route] = 1.0f;
+  if (smask) atomicOr(&smask[d.E_route], 1u << warp);
+}
+
 template <int PER>
 __global__ void __launch_bounds__(256)
 route_kernel(const float* __restrict__ logits, Dims d, Work w) {
@@ -117,9 +127,11 @@ route_kernel(const float* __restrict__ logits, Dims d, Work w) {
   }
   for (int e = threadIdx.x; e < d.E; e += blockDim.x) smask[e] = 0u;
   __syncthreads();
-  if (t < d.T)
-    route_token<PER>(logits + (size_t)t * d.E, d.E, d.k, lane, w.idx + (size_t)t * d.k, w.pw + (size_t)t * d.k,
-                     [&](int e) { atomicOr(&smask[e], 1u << warp); });
+  if (t < d.T) {
+    route_token<PER>(logits + (size_t)t * d.E_route, d.E_route, d.k_route, lane, w.idx + (size_t)t * d.k,
+                     w.pw + (size_t)t * d.k, [&](int e) { atomicOr(&smask[e], 1u << warp); });
+    if (d.k > d.k_route && lane == 0) append_shared(d, w.idx + (size_t)t * d.k, w.pw + (size_t)t * d.k, smask, warp);
+  }
   __syncthreads();
   uint8_t* bm8 = reinterpret_cast<uint8_t*>(w.bitmap);
   const size_t row_bytes = (size_t)d.W * 4;

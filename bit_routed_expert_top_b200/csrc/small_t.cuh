@@ -160,7 +160,8 @@ gateup_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ lo
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int G = Fmt<FMT>::kGroup;
   if (warp == 0) {
-    route_token<PER>(logits + (size_t)t * d.E, d.E, d.k, lane, s_idx, s_pw, [](int) {});
+    route_token<PER>(logits + (size_t)t * d.E_route, d.E_route, d.k_route, lane, s_idx, s_pw, [](int) {});
+    if (d.k > d.k_route && lane == 0) append_shared(d, s_idx, s_pw, nullptr, 0);
   } else {
     // x_t -> fp16 (one rounding from the exact bf16 value, as the prefill
     // path stages it) in the decoder's K order: word v of the row holds

@@ -132,6 +132,31 @@ int rl_moe_prefill_ws(const void* x, const float* router_logits,
                       int I, int E, int k, float* y, void* workspace,
                       size_t ws_bytes, void* stream);
 
+/* Workspace bytes rl_moe_prefill_shared_ws needs (E + 1 experts, k + 1
+ * picks per token); 0 on a bad argument (E + 1 must not exceed
+ * RL_MAX_EXPERTS). */
+size_t rl_moe_shared_workspace_bytes(int fmt, int T, int H, int I, int E, int k);
+
+/* The layer with a shared expert upstream of the routed sum, fused with the
+ * routing step: every token's selection gets one more pick, the shared
+ * expert, after its k routed picks and with weight 1, so that
+ *   y[t] = sum_{j<k} p_{t,j} o_{t,j} + s_t,  s_t = W_down(silu(W_gate x_t) *
+ *   W_up x_t) of the shared expert,
+ * added in that order in fp32.  "Red Lite dev75 - --kv f16, faster prompt
+ * ingestion", section 2, lists a shared expert beside the routed experts in
+ * the prefill and gives it no size, format or gate: here it has the routed
+ * experts' block format and shape and no gate.
+ *   shared_blob  device pointer, 16-byte aligned, rl_moe_expert_bytes(fmt,
+ *                H, I) long.
+ *   workspace    at least rl_moe_shared_workspace_bytes() bytes, 256-byte
+ *                aligned.
+ * Every other argument, the status word and the ordering rules as for
+ * rl_moe_prefill_ws (E routed experts, router_logits [T, E]). */
+int rl_moe_prefill_shared_ws(const void* x, const float* router_logits,
+                             const void* const* expert_blobs, const void* shared_blob,
+                             int fmt, int T, int H, int I, int E, int k, float* y,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /*
  * The router projection upstream of step 1 ("Red Lite dev72 - bounded
  * verify, profiling", section 1: the router runs per row before the
