@@ -405,6 +405,50 @@ def router_gemm_figure(args, dev, flush, wl):
                                    "grouping, decode-GEMMs, combine); median of the timed steps"}
 
 
+def shared_expert_figure(args, dev, flush, wl):
+    """The layer with a shared expert (rl_moe_prefill_shared_ws: every token
+    picks the shared expert last, weight 1) at the workload's shape, the
+    shared blob at the routed experts' stride: median ms over the timed
+    steps (L2 flushed before each), pairs/s over T*(k+1) pairs and the
+    fraction of its roofline (FLOPs and bytes of k+1 picks per token)."""
+    import torch
+    from bit_routed_expert_top_b200 import api
+
+    peaks, _ = load_peaks()
+    wl1 = synth.Workload(wl.name, wl.T, wl.H, wl.I, wl.E + 1, wl.k, wl.fmt, wl.skew)
+    inp = synth.make_inputs(wl1)
+    x = torch.from_numpy(inp.x_bits.view(np.int16).copy()).to(dev)
+    logits = torch.from_numpy(np.ascontiguousarray(inp.logits[:, :wl.E])).to(dev)
+    blobs = torch.from_numpy(inp.blobs).to(dev)
+    table = api.expert_table(blobs, wl.E)
+    y = torch.empty((wl.T, wl.H), dtype=torch.float32, device=dev)
+    ws = api.alloc_shared_workspace(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.warmup):
+        flush.fill_(float(i))
+        api.rl_moe_prefill_shared_ws(x, logits, table, blobs[wl.E], wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws)
+    for i, (a, b) in enumerate(ev):
+        flush.fill_(float(i))
+        a.record(stream)
+        api.rl_moe_prefill_shared_ws(x, logits, table, blobs[wl.E], wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, y, ws)
+        b.record(stream)
+    torch.cuda.synchronize()
+    if api.rl_moe_check_status(ws) != 0:
+        raise RuntimeError("shared-expert layer: device status " + api.rl_last_error())
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    top = np.argsort(-inp.logits[:, :wl.E], axis=1, kind="stable")[:, :wl.k]
+    touched = int(np.unique(top).size) + 1
+    wlk = synth.Workload(wl.name, wl.T, wl.H, wl.I, wl.E, wl.k + 1, wl.fmt, wl.skew)
+    model = layer_model(wlk, touched)
+    t_roof = max(model["flops"] / (peaks["bf16_tflops"] * 1e12), model["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    P = wl.T * (wl.k + 1)
+    return {"T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "pairs": P, "ms_median": ms,
+            "pairs_per_s": P / (ms * 1e-3), "t_roof_ms": t_roof, "layer_roofline_frac": t_roof / ms,
+            "method": "rl_moe_prefill_shared_ws, the shared blob at the routed experts' stride; median of the "
+                      "timed steps, L2 flushed before each"}
+
+
 def bench_ours(args, wl, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -558,9 +602,11 @@ def bench_ours(args, wl, world, rank, local):
         del graph
     per_wl = None
     router = None
+    shared = None
     if world == 1 and not args.no_per_workload:
         per_wl = per_workload_figures(args, dev, flush, wl.name)
         router = router_gemm_figure(args, dev, flush, wl)
+        shared = shared_expert_figure(args, dev, flush, wl)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -620,6 +666,8 @@ def bench_ours(args, wl, world, rank, local):
         line["per_workload"] = per_wl
     if router is not None:
         line["router_gemm"] = router
+    if shared is not None:
+        line["shared_expert"] = shared
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)
