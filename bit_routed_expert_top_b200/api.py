@@ -49,6 +49,8 @@ SIGNATURES = {
     "rl_moe_router_logits": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
     "rl_moe_router_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "rl_moe_prefill_router_ws": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "rl_moe_router_shared_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "rl_moe_prefill_router_shared_ws": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
 }
 RL_CACHE_HOST_POOL = 0x1
 # Not in the public header: selects the CUDA-core decode-GEMMs for stage-by-
@@ -347,6 +349,30 @@ def rl_moe_prefill_router_ws(x, w_router, expert_blobs, fmt, T, H, I, E, k, y, w
     nbytes = workspace.numel() * workspace.element_size()
     _check(load().rl_moe_prefill_router_ws(_ptr(x), _ptr(w_router), ctypes.cast(table, ctypes.c_void_p), fmt, T, H,
                                            I, E, k, _ptr(y), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def rl_moe_router_shared_workspace_bytes(fmt: int, T: int, H: int, I: int, E: int, k: int) -> int:
+    n = load().rl_moe_router_shared_workspace_bytes(fmt, T, H, I, E, k)
+    if n == 0:
+        raise RlMoeError(-1, load().rl_last_error().decode(errors="replace"))
+    return n
+
+
+def rl_moe_prefill_router_shared_ws(x, w_router, expert_blobs, shared_blob, fmt, T, H, I, E, k, y, workspace,
+                                    stream=None):
+    """Router GEMM, then the layer with the shared expert as every token's
+    last pick; see include/rl_moe.h."""
+    _check_buf(x, "x", _X_DTYPES, T * H)
+    _check_buf(w_router, "w_router", _X_DTYPES, E * H)
+    _check_buf(y, "y", (torch.float32,), T * H)
+    _check_buf(shared_blob, "shared_blob", (torch.uint8,), rl_moe_expert_bytes(fmt, H, I))
+    _check_buf(workspace, "workspace", (), 0)
+    _need_cuda(x, w_router, y, workspace, shared_blob)
+    table = expert_blobs if isinstance(expert_blobs, ctypes.Array) else expert_table(expert_blobs, E)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load().rl_moe_prefill_router_shared_ws(_ptr(x), _ptr(w_router), ctypes.cast(table, ctypes.c_void_p),
+                                                  _ptr(shared_blob), fmt, T, H, I, E, k, _ptr(y), _ptr(workspace),
+                                                  nbytes, _stream(stream)))
 
 
 def rl_moe_check_status(workspace, stream=None) -> int:

@@ -559,24 +559,30 @@ size_t rl_moe_router_workspace_bytes(int fmt, int T, int H, int I, int E, int k)
   return n ? n + align_up((size_t)T * E * 4, 256) : 0;
 }
 
-int rl_moe_prefill_router_ws(const void* x, const void* w_router, const void* const* expert_blobs, int fmt, int T,
-                             int H, int I, int E, int k, float* y, void* workspace, size_t ws_bytes,
-                             void* stream) {
+// Router GEMM, then the layer from its logits; with shared_blob (not null)
+// the shared expert is every token's last pick.
+static int router_layer_ws(const void* x, const void* w_router, const void* const* expert_blobs,
+                           const void* shared_blob, int fmt, int T, int H, int I, int E, int k, float* y,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  const int shared = shared_blob ? 1 : 0;
   rl::Dims d;
   Layout L;
-  int rc = plan(fmt, T, H, I, E, k, &d, &L);
+  int rc = plan(fmt, T, H, I, E, k, &d, &L, shared);
   if (rc != RL_OK) return rc;
   if (T == 0) return RL_OK;
   if (!x || !w_router || !y || !workspace)
     return fail(RL_ERR_INVALID_ARG, "NULL x, w_router, y or workspace");
   if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(w_router) % 16 ||
-      reinterpret_cast<uintptr_t>(y) % 16 || reinterpret_cast<uintptr_t>(workspace) % 256)
-    return fail(RL_ERR_INVALID_ARG, "x, w_router and y must be 16-byte aligned, workspace 256-byte aligned");
+      reinterpret_cast<uintptr_t>(y) % 16 || reinterpret_cast<uintptr_t>(workspace) % 256 ||
+      reinterpret_cast<uintptr_t>(shared_blob) % 16)
+    return fail(RL_ERR_INVALID_ARG,
+                "x, w_router, y and shared_blob must be 16-byte aligned, workspace 256-byte aligned");
   const size_t need = L.total + align_up((size_t)T * E * 4, 256);
   if (ws_bytes < need) return fail(RL_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, need);
   static thread_local rl::ExpertTable tab;
   rc = fill_table(expert_blobs, E, &tab);
   if (rc != RL_OK) return rc;
+  if (shared) tab.p[E] = static_cast<const uint8_t*>(shared_blob);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const rl::Work w = carve(workspace, L);
   float* logits = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.total);
@@ -593,6 +599,25 @@ int rl_moe_prefill_router_ws(const void* x, const void* w_router, const void* co
   }
   return fmt == RL_FMT_Q2 ? launch_all<RL_FMT_Q2>(x, logits, tab, d, w, y, s)
                           : launch_all<RL_FMT_Q1>(x, logits, tab, d, w, y, s);
+}
+
+int rl_moe_prefill_router_ws(const void* x, const void* w_router, const void* const* expert_blobs, int fmt, int T,
+                             int H, int I, int E, int k, float* y, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  return router_layer_ws(x, w_router, expert_blobs, nullptr, fmt, T, H, I, E, k, y, workspace, ws_bytes, stream);
+}
+
+size_t rl_moe_router_shared_workspace_bytes(int fmt, int T, int H, int I, int E, int k) {
+  const size_t n = rl_moe_shared_workspace_bytes(fmt, T, H, I, E, k);
+  return n ? n + align_up((size_t)T * E * 4, 256) : 0;
+}
+
+int rl_moe_prefill_router_shared_ws(const void* x, const void* w_router, const void* const* expert_blobs,
+                                    const void* shared_blob, int fmt, int T, int H, int I, int E, int k, float* y,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  if (!shared_blob) return fail(RL_ERR_INVALID_ARG, "shared_blob is NULL");
+  return router_layer_ws(x, w_router, expert_blobs, shared_blob, fmt, T, H, I, E, k, y, workspace, ws_bytes,
+                         stream);
 }
 
 int rl_moe_prefill(const void* x, const float* router_logits, const void* const* expert_blobs,

@@ -186,6 +186,21 @@ int rl_moe_prefill_router_ws(const void* x, const void* w_router, const void* co
                              int fmt, int T, int H, int I, int E, int k, float* y, void* workspace,
                              size_t ws_bytes, void* stream);
 
+/* Workspace bytes rl_moe_prefill_router_shared_ws needs; 0 on a bad
+ * argument. */
+size_t rl_moe_router_shared_workspace_bytes(int fmt, int T, int H, int I, int E, int k);
+
+/* The router GEMM and the shared expert upstream of the path, fused with the
+ * routing step: the router projection (as rl_moe_prefill_router_ws), then
+ * the layer from its logits with the shared expert as every token's last
+ * pick (as rl_moe_prefill_shared_ws; same reading of "Red Lite dev75 - --kv
+ * f16, faster prompt ingestion", section 2).  shared_blob must not be NULL;
+ * workspace at least rl_moe_router_shared_workspace_bytes() bytes. */
+int rl_moe_prefill_router_shared_ws(const void* x, const void* w_router,
+                                    const void* const* expert_blobs, const void* shared_blob,
+                                    int fmt, int T, int H, int I, int E, int k, float* y,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
 /* Fixed size of the scratch array used by rl_moe_prefill_noalloc (16 MiB). */
 #define RL_NOALLOC_SCRATCH_BYTES (16u << 20)
 

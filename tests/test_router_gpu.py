@@ -167,3 +167,30 @@ def test_layer_from_x_equals_routing_the_exported_logits(T, H, I, E, k, ties):
         for t in range(T):
             if 130 in idx[t]:
                 assert 3 in idx[t] and list(idx[t]).index(3) < list(idx[t]).index(130)
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [(300, 256, 256, 96, 6), (2, 2048, 512, 512, 10)],
+                         ids=["prefill_path", "decode_regime"])
+def test_router_and_shared_expert_equal_the_two_step_calls(T, H, I, E, k):
+    """Router GEMM + layer with the shared expert in one call: y equals, bit
+    for bit, rl_moe_prefill_shared_ws on the logits rl_moe_router_logits
+    returns for the same x and W_r."""
+    wl = synth.Workload("fused_shared", T, H, I, E + 1, k, synth.FMT_Q2)
+    inp = synth.make_inputs(wl, seed=41)
+    w = synth.router_weights(E, H, seed=42)
+    x = torch.from_numpy(inp.x_bits.view(np.int16).copy()).cuda()
+    blobs = torch.from_numpy(inp.blobs).cuda()
+    table = api.expert_table(blobs, E)
+    wd = torch.from_numpy(w.view(np.int16).copy()).cuda()
+    y = torch.full((T, H), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(api.rl_moe_router_shared_workspace_bytes(wl.fmt, T, H, I, E, k), dtype=torch.uint8,
+                     device="cuda")
+    api.rl_moe_prefill_router_shared_ws(x, wd, table, blobs[E], wl.fmt, T, H, I, E, k, y, ws)
+    assert api.rl_moe_check_status(ws) == 0, api.rl_last_error()
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    api.rl_moe_router_logits(x, wd, T, H, E, logits)
+    y_ref = torch.full_like(y, float("nan"))
+    ws2 = api.alloc_shared_workspace(wl.fmt, T, H, I, E, k)
+    api.rl_moe_prefill_shared_ws(x, logits, table, blobs[E], wl.fmt, T, H, I, E, k, y_ref, ws2)
+    assert api.rl_moe_check_status(ws2) == 0, api.rl_last_error()
+    assert torch.equal(y, y_ref)
