@@ -449,6 +449,78 @@ def shared_expert_figure(args, dev, flush, wl):
                       "timed steps, L2 flushed before each"}
 
 
+def expert_cache_figure(args, dev, flush):
+    """Bounded verify steps (rl_moe_verify_bounded) at the 2-token verify
+    shape on a cache of 64 of the 512 experts filled from pinned host memory:
+    per step new router logits (new selections: misses are copied host ->
+    device inside the step) and, separately, steps that repeat the previous
+    step's selections (every expert resident).  Device time per step (CUDA
+    events; the step reads its selections back to the host in between),
+    misses and bytes copied per step, and a plain pinned host -> device copy
+    of 64 MB as the copy bandwidth reference."""
+    import torch
+    from bit_routed_expert_top_b200 import api
+
+    wl = [w for w in synth.WORKLOADS if w.name == "verify2"][0]
+    base = synth.make_inputs(wl)
+    host = torch.from_numpy(base.blobs).pin_memory()
+    cache = api.ExpertCache(wl.fmt, wl.H, wl.I, wl.E, 64, host)
+    ws = api.alloc_workspace(wl.fmt, wl.T, wl.H, wl.I, wl.E, wl.k, device=dev)
+    rng = np.random.default_rng(13)
+    stream = torch.cuda.current_stream(dev)
+    y = torch.empty((wl.T, wl.H), dtype=torch.float32, device=dev)
+    x = torch.from_numpy(synth.f32_to_bf16_bits(rng.standard_normal((wl.T, wl.H), dtype=np.float32))
+                         .view(np.int16).copy()).to(dev)
+
+    def steps(n, fresh):
+        times, misses, copied = [], [], []
+        logits = torch.from_numpy(rng.standard_normal((wl.T, wl.E), dtype=np.float32)).to(dev)
+        for i in range(n):
+            if fresh:
+                logits = torch.from_numpy(rng.standard_normal((wl.T, wl.E), dtype=np.float32)).to(dev)
+            flush.fill_(float(i))
+            st0 = cache.stats()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            api.rl_moe_verify_bounded(cache, x, logits, wl.T, wl.k, y, ws)
+            b.record(stream)
+            b.synchronize()
+            st1 = cache.stats()
+            times.append(a.elapsed_time(b))
+            misses.append(st1["misses"] - st0["misses"])
+            copied.append(st1["bytes_copied"] - st0["bytes_copied"])
+        return times, misses, copied
+
+    steps(args.warmup, True)
+    t_miss, m_miss, b_miss = steps(args.steps, True)
+    t_hit, m_hit, _ = steps(args.steps, False)
+    if api.rl_moe_check_status(ws) != 0:
+        raise RuntimeError("bounded verify: device status " + api.rl_last_error())
+    # pinned host -> device copy bandwidth on the same stream
+    src = torch.empty(64 << 20, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
+    dst.copy_(src, non_blocking=True)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(4):
+        dst.copy_(src, non_blocking=True)
+    b.record(stream)
+    b.synchronize()
+    h2d_gbs = 4 * (64 << 20) / (a.elapsed_time(b) * 1e-3) / 1e9
+    cache.close()
+    med_miss = statistics.median(t_miss)
+    bytes_med = statistics.median(b_miss)
+    return {"shape": "verify2 (T=2, H=2048, I=512, E=512, k=10, Q2)", "slots": 64,
+            "ms_median_new_selections": med_miss, "misses_median": statistics.median(m_miss),
+            "bytes_copied_median": bytes_med,
+            "copy_gbs_effective": bytes_med / (med_miss * 1e-3) / 1e9 if med_miss else None,
+            "ms_median_resident": statistics.median(t_hit), "misses_resident": int(sum(m_hit)),
+            "h2d_pinned_gbs": h2d_gbs,
+            "method": "rl_moe_verify_bounded per step (selections read back to the host inside the step), "
+                      "CUDA events on the stream, L2 flushed before each; steps with new router logits "
+                      "(misses copied inside the step) and steps repeating the previous logits"}
+
+
 def bench_ours(args, wl, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -603,10 +675,12 @@ def bench_ours(args, wl, world, rank, local):
     per_wl = None
     router = None
     shared = None
+    cache_fig = None
     if world == 1 and not args.no_per_workload:
         per_wl = per_workload_figures(args, dev, flush, wl.name)
         router = router_gemm_figure(args, dev, flush, wl)
         shared = shared_expert_figure(args, dev, flush, wl)
+        cache_fig = expert_cache_figure(args, dev, flush)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -668,6 +742,8 @@ def bench_ours(args, wl, world, rank, local):
         line["router_gemm"] = router
     if shared is not None:
         line["shared_expert"] = shared
+    if cache_fig is not None:
+        line["expert_cache"] = cache_fig
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)
