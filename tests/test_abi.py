@@ -177,3 +177,31 @@ def test_fault_switch_accepts_only_known_bits():
     assert lib.rl_moe_debug_set_fault(0x10, 0) == -1        # RL_ERR_INVALID_ARG
     assert lib.rl_moe_debug_set_fault(1, 2_000_000) == 0
     assert lib.rl_moe_debug_set_fault(0, 0) == 0
+
+
+def test_shared_expert_entries_validate_on_the_host():
+    """The shared-expert entries: workspace sizes are those of E + 1 experts
+    and k + 1 picks; a NULL or misaligned shared blob, a short workspace and
+    E + 1 beyond the expert limit are refused before any CUDA call."""
+    lib = api.load()
+    for fmt, T, H, I, E, k in [(2, 2048, 2048, 512, 512, 10), (1, 2, 512, 256, 64, 8)]:
+        assert api.rl_moe_shared_workspace_bytes(fmt, T, H, I, E, k) == api.rl_moe_workspace_bytes(
+            fmt, T, H, I, E + 1, k + 1)
+        assert api.rl_moe_router_shared_workspace_bytes(fmt, T, H, I, E, k) == (
+            api.rl_moe_shared_workspace_bytes(fmt, T, H, I, E, k) + (T * E * 4 + 255) // 256 * 256)
+    assert lib.rl_moe_shared_workspace_bytes(2, 8, 256, 128, 1024, 2) == 0      # E + 1 > 1024
+    assert lib.rl_moe_shared_workspace_bytes(2, 8, 256, 128, 1023, 2) > 0
+    tab = (ctypes.c_void_p * 16)(*([0x1000] * 16))
+    t = ctypes.cast(tab, ctypes.c_void_p)
+    rc = lib.rl_moe_prefill_shared_ws(0x1000, 0x1000, t, None, 2, 8, 256, 128, 16, 2, 0x1000, 0x1000, 1 << 30, None)
+    assert rc == -1 and "NULL" in api.rl_last_error()
+    rc = lib.rl_moe_prefill_shared_ws(0x1000, 0x1000, t, 0x1008, 2, 8, 256, 128, 16, 2, 0x1000, 0x1000, 1 << 30,
+                                      None)
+    assert rc == -1 and "aligned" in api.rl_last_error()
+    need = api.rl_moe_shared_workspace_bytes(2, 8, 256, 128, 16, 2)
+    rc = lib.rl_moe_prefill_shared_ws(0x1000, 0x1000, t, 0x1000, 2, 8, 256, 128, 16, 2, 0x1000, 0x1000, need - 256,
+                                      None)
+    assert rc == -1 and "workspace" in api.rl_last_error()
+    rc = lib.rl_moe_prefill_router_shared_ws(0x1000, 0x1000, t, None, 2, 8, 256, 128, 16, 2, 0x1000, 0x1000,
+                                             1 << 30, None)
+    assert rc == -1 and "NULL" in api.rl_last_error()
