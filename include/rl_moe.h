@@ -21,6 +21,13 @@
  *   5. combine  y[t] = sum_j p_j o_{t,j}, added in selection order
  *               (dev75 section 3: the MoE tail sums in selection order).
  *
+ * Around it: the router projection upstream of step 1 (rl_moe_router_logits,
+ * rl_moe_prefill_router_ws), a shared expert fused with step 1 as every
+ * token's last pick with weight 1 (rl_moe_prefill_shared_ws,
+ * rl_moe_prefill_router_shared_ws), a decode regime for chunks of at most 64
+ * pairs (taken by the same entry points), and a bounded expert cache
+ * (rl_moe_cache_*, rl_moe_verify_bounded).
+ *
  * Weight formats (stand-ins for IQ2_XS / IQ1_M, whose grids the pages do not
  * print).  A block holds 256 consecutive values of one row along K:
  *   RL_FMT_Q2, 69 bytes: [0,2) fp16 d (little endian); [2,5) 24-bit LE word,
