@@ -105,6 +105,7 @@ DECODE = [
     synth.Workload("sh_t1", 1, 2048, 512, 512, 10, synth.FMT_Q2),
     synth.Workload("sh_t2", 2, 2048, 512, 512, 10, synth.FMT_Q2),
     synth.Workload("sh_t2_q1", 2, 1024, 512, 64, 8, synth.FMT_Q1),
+    synth.Workload("sh_e1023", 2, 512, 256, 1023, 8, synth.FMT_Q1),   # E + 1 = 1024, the expert limit
 ]
 
 
